@@ -1,0 +1,16 @@
+"""fp64 CPU oracle (test infrastructure only; never on the product path).
+
+Only the tests, the package smoke check and the benchmark's CPU-baseline leg
+may import this package.
+"""
+from .ssa_oracle import (  # noqa: F401
+    attention_probs,
+    block_summary,
+    decode,
+    decode_route,
+    pool_query_blocks,
+    route,
+    select_topk,
+    sparse_attention,
+    summary_scores,
+)
