@@ -1,0 +1,210 @@
+"""ctypes binding of ``libssa.so`` (argument marshalling only).
+
+Every function here has the name of the C entry point it calls, takes torch
+CUDA tensors, passes their device pointers and the current CUDA stream, and
+raises ``SSAError`` on a non-OK status.  Outputs that the caller does not
+pass are allocated with torch (device memory is torch's job; the library
+allocates nothing).  No step of the method runs here.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libssa.so")
+
+SSA_F32 = 0
+SSA_BF16 = 1
+
+_STATUS = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED", 3: "SSA_ERR_CUDA",
+           4: "SSA_ERR_TIMEOUT"}
+
+# Every symbol include/ssa.h declares.
+EXPORTS = ("ssa_status_string", "ssa_version", "ssa_block_summary", "ssa_route",
+           "ssa_sparse_attn_fwd", "ssa_sparse_attn_uses_tensor_cores", "ssa_decode_workspace_size",
+           "ssa_decode", "ssa_device_error")
+
+
+class SSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {_STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load (once) and return the library.  Raises if it was not built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(
+            f"libssa.so not found at {p}: build it with "
+            "`python -m block_sparse_top_summary_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(p)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.ssa_status_string.restype = ctypes.c_char_p
+    lib.ssa_status_string.argtypes = [i]
+    lib.ssa_version.restype = i
+    lib.ssa_block_summary.argtypes = [vp, i, i, i, i, i, i, vp, vp]
+    lib.ssa_route.argtypes = [vp, i, vp, i, i, i, i, i, i, i, i, vp, vp, vp]
+    lib.ssa_sparse_attn_fwd.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp]
+    lib.ssa_decode_workspace_size.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(sz)]
+    lib.ssa_decode.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, sz, vp]
+    lib.ssa_device_error.argtypes = [ctypes.POINTER(i)]
+    lib.ssa_sparse_attn_uses_tensor_cores.argtypes = [i, i, i, i, i]
+    for name in EXPORTS:
+        if name not in ("ssa_status_string", "ssa_version"):
+            getattr(lib, name).restype = i
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise SSAError(fn, status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SSA_F32
+    if t.dtype == torch.bfloat16:
+        return SSA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def ssa_block_summary(K: torch.Tensor, B: int, S: torch.Tensor | None = None, stream=None):
+    """Block mean summaries ``S`` ``[batch, Hkv, N // B, d]`` fp32 of ``K``."""
+    _need(K, "K")
+    batch, Hkv, N, d = K.shape
+    if S is None:
+        S = torch.empty(batch, Hkv, N // B, d, dtype=torch.float32, device=K.device)
+    _check("ssa_block_summary", load_library().ssa_block_summary(
+        _ptr(K), _dtype_code(K), batch, Hkv, N, d, B, _ptr(S), _stream(stream)))
+    return S
+
+
+def route_width(N: int, B: int, topk: int) -> int:
+    """Smallest idx row width for ssa_route."""
+    nq = -(-N // B)
+    return min(topk, max(nq - 2, 0)) + 2
+
+
+def ssa_route(Q: torch.Tensor, S: torch.Tensor, B: int, topk: int, Hkv: int,
+              max_sel: int | None = None, idx=None, cnt=None, stream=None):
+    """Top-k routing per (batch, KV head, query block): returns ``(idx, cnt)``."""
+    _need(Q, "Q")
+    batch, Hq, N, d = Q.shape
+    nq = -(-N // B)
+    if max_sel is None:
+        max_sel = route_width(N, B, topk)
+    if idx is None:
+        idx = torch.empty(batch, Hkv, nq, max_sel, dtype=torch.int32, device=Q.device)
+    if cnt is None:
+        cnt = torch.empty(batch, Hkv, nq, dtype=torch.int32, device=Q.device)
+    _check("ssa_route", load_library().ssa_route(
+        _ptr(Q), _dtype_code(Q), _ptr(S), batch, Hq, Hkv, N, d, B, topk, max_sel, _ptr(idx),
+        _ptr(cnt), _stream(stream)))
+    return idx, cnt
+
+
+def ssa_sparse_attn_fwd(Q, K, V, idx, cnt, B: int, scale: float | None = None, O=None, lse=None,
+                        want_lse: bool = True, stream=None):
+    """Attention over the selected blocks: returns ``(O, lse)`` (``lse`` may be None)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (idx, "idx"), (cnt, "cnt")):
+        _need(t, n)
+    batch, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty(batch, Hq, N, dtype=torch.float32, device=Q.device)
+    _check("ssa_sparse_attn_fwd", load_library().ssa_sparse_attn_fwd(
+        _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(idx), _ptr(cnt), batch, Hq, Hkv, N, d, B,
+        idx.shape[-1], ctypes.c_float(scale), _ptr(O), _ptr(lse), _stream(stream)))
+    return O, lse
+
+
+def ssa_sparse_attn_uses_tensor_cores(dtype: torch.dtype, Hq: int, Hkv: int, d: int,
+                                      B: int) -> bool:
+    code = SSA_BF16 if dtype == torch.bfloat16 else SSA_F32
+    return bool(load_library().ssa_sparse_attn_uses_tensor_cores(code, Hq, Hkv, d, B))
+
+
+def ssa_decode_workspace_size(batch: int, Hq: int, Hkv: int, Lmax: int, d: int, B: int,
+                              topk: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ssa_decode_workspace_size", load_library().ssa_decode_workspace_size(
+        batch, Hq, Hkv, Lmax, d, B, topk, ctypes.byref(n)))
+    return n.value
+
+
+def decode_width(Lmax: int, B: int, topk: int) -> int:
+    return min(topk, -(-Lmax // B)) + 2
+
+
+def ssa_decode(q, Kc, Vc, S, seqlens, B: int, topk: int, scale: float | None = None, O=None,
+               idx=None, want_idx: bool = True, workspace=None, stream=None):
+    """One decode step: returns ``(O, idx)`` (``idx`` None unless wanted)."""
+    for t, n in ((q, "q"), (Kc, "Kc"), (Vc, "Vc"), (seqlens, "seqlens")):
+        _need(t, n)
+    batch, Hq, d = q.shape
+    Hkv, Lmax = Kc.shape[1], Kc.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(q)
+    if idx is None and want_idx:
+        idx = torch.empty(batch, Hkv, decode_width(Lmax, B, topk), dtype=torch.int32,
+                          device=q.device)
+    ws_bytes = ssa_decode_workspace_size(batch, Hq, Hkv, Lmax, d, B, topk)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check("ssa_decode", load_library().ssa_decode(
+        _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(S), _ptr(seqlens), batch, Hq, Hkv, Lmax,
+        d, B, topk, ctypes.c_float(scale), _ptr(O), _ptr(idx), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return O, idx
+
+
+def ssa_device_error() -> int:
+    """Synchronise, then read and reset the device-side error word."""
+    code = ctypes.c_int(0)
+    _check("ssa_device_error", load_library().ssa_device_error(ctypes.byref(code)))
+    return code.value
+
+
+def prefill(Q, K, V, B: int, topk: int, scale: float | None = None, stream=None):
+    """The three prefill calls in order: summary, route, attention.
+
+    Returns ``(O, lse, idx, cnt, S)``.
+    """
+    S = ssa_block_summary(K, B, stream=stream)
+    idx, cnt = ssa_route(Q, S, B, topk, K.shape[1], stream=stream)
+    O, lse = ssa_sparse_attn_fwd(Q, K, V, idx, cnt, B, scale=scale, stream=stream)
+    return O, lse, idx, cnt, S

@@ -1,0 +1,144 @@
+// C ABI entry points: host-side argument checks, then the kernel launches.
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "ssa.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dtype_ok(ssa_dtype dt) { return dt == SSA_F32 || dt == SSA_BF16; }
+
+// Shape checks shared by every entry point.  Returns SSA_OK or the error.
+ssa_status check_dims(int d, int B, ssa_dtype dt) {
+  if (!dtype_ok(dt)) return SSA_ERR_INVALID_ARG;
+  if (B <= 0 || d <= 0) return SSA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SSA_ERR_UNSUPPORTED;
+  if (B % 16 != 0 || B > 128) return SSA_ERR_UNSUPPORTED;
+  return SSA_OK;
+}
+
+ssa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* ssa_status_string(int status) {
+  switch (status) {
+    case SSA_OK: return "SSA_OK";
+    case SSA_ERR_INVALID_ARG: return "SSA_ERR_INVALID_ARG";
+    case SSA_ERR_UNSUPPORTED: return "SSA_ERR_UNSUPPORTED";
+    case SSA_ERR_CUDA: return "SSA_ERR_CUDA";
+    case SSA_ERR_TIMEOUT: return "SSA_ERR_TIMEOUT";
+    default: return "SSA_ERR_UNKNOWN";
+  }
+}
+
+int ssa_version(void) { return 100; }
+
+ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv, int N, int d,
+                             int B, float* S, ssa_stream stream) {
+  ssa_status st = check_dims(d, B, dtype);
+  if (st != SSA_OK) return st;
+  if (batch <= 0 || Hkv <= 0 || N <= 0) return SSA_ERR_INVALID_ARG;
+  if (N / B == 0) return SSA_OK;
+  if (K == nullptr || S == nullptr) return SSA_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(S)) return SSA_ERR_INVALID_ARG;
+  return from_cuda(ssa::launch_block_summary(K, dtype, batch, Hkv, N, d, B, S,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ssa_status ssa_route(const void* Q, ssa_dtype dtype, const float* S, int batch, int Hq, int Hkv,
+                     int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
+                     ssa_stream stream) {
+  ssa_status st = check_dims(d, B, dtype);
+  if (st != SSA_OK) return st;
+  if (batch <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || topk < 0) return SSA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
+  const int nq = (N + B - 1) / B;
+  if (nq > ssa::kRouteMaxBlocks) return SSA_ERR_UNSUPPORTED;
+  const int cand_max = nq > 2 ? nq - 2 : 0;
+  const int need = (topk < cand_max ? topk : cand_max) + 2;
+  if (max_sel < need) return SSA_ERR_INVALID_ARG;
+  if (Q == nullptr || idx == nullptr || cnt == nullptr) return SSA_ERR_INVALID_ARG;
+  if (N / B > 0 && S == nullptr) return SSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(S)) return SSA_ERR_INVALID_ARG;
+  return from_cuda(ssa::launch_route(Q, dtype, S, batch, Hq, Hkv, N, d, B, topk, max_sel, idx, cnt,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ssa_status ssa_sparse_attn_fwd(const void* Q, const void* K, const void* V, ssa_dtype dtype,
+                               const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
+                               int N, int d, int B, int max_sel, float scale, void* O, float* lse,
+                               ssa_stream stream) {
+  ssa_status st = check_dims(d, B, dtype);
+  if (st != SSA_OK) return st;
+  if (batch <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || max_sel < 1) return SSA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return SSA_ERR_INVALID_ARG;
+  if (Q == nullptr || K == nullptr || V == nullptr || idx == nullptr || cnt == nullptr ||
+      O == nullptr)
+    return SSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return SSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (ssa::attn_tc_supported(dtype, Hq, Hkv, d, B))
+    return from_cuda(
+        ssa::launch_attn_tc(Q, K, V, idx, cnt, batch, Hq, Hkv, N, B, max_sel, scale, O, lse, s));
+  return from_cuda(ssa::launch_attn_simt(Q, K, V, dtype, idx, cnt, batch, Hq, Hkv, N, d, B,
+                                         max_sel, scale, O, lse, s));
+}
+
+int ssa_sparse_attn_uses_tensor_cores(ssa_dtype dtype, int Hq, int Hkv, int d, int B) {
+  if (!dtype_ok(dtype) || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
+  return ssa::attn_tc_supported(dtype, Hq, Hkv, d, B) ? 1 : 0;
+}
+
+ssa_status ssa_decode_workspace_size(int batch, int Hq, int Hkv, int Lmax, int d, int B, int topk,
+                                     size_t* bytes) {
+  if (bytes == nullptr) return SSA_ERR_INVALID_ARG;
+  ssa_status st = check_dims(d, B, SSA_BF16);
+  if (st != SSA_OK) return st;
+  if (batch <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || topk < 0) return SSA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
+  *bytes = ssa::plan_decode(batch, Hq, Hkv, d, B, topk, Lmax).bytes;
+  return SSA_OK;
+}
+
+ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype dtype,
+                      const float* S, const int32_t* seqlens, int batch, int Hq, int Hkv, int Lmax,
+                      int d, int B, int topk, float scale, void* O, int32_t* idx, void* workspace,
+                      size_t ws_bytes, ssa_stream stream) {
+  ssa_status st = check_dims(d, B, dtype);
+  if (st != SSA_OK) return st;
+  if (batch <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || topk < 0) return SSA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
+  if (Hq / Hkv > 8) return SSA_ERR_UNSUPPORTED;
+  if (Lmax / B > 16384) return SSA_ERR_UNSUPPORTED;
+  if (!(scale > 0.f)) return SSA_ERR_INVALID_ARG;
+  if (q == nullptr || Kc == nullptr || Vc == nullptr || seqlens == nullptr || O == nullptr ||
+      workspace == nullptr)
+    return SSA_ERR_INVALID_ARG;
+  if (Lmax / B > 0 && S == nullptr) return SSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(S) || !aligned16(O))
+    return SSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSA_ERR_INVALID_ARG;
+  const ssa::DecodePlan p = ssa::plan_decode(batch, Hq, Hkv, d, B, topk, Lmax);
+  if (ws_bytes < p.bytes) return SSA_ERR_INVALID_ARG;
+  return from_cuda(ssa::launch_decode(p, q, Kc, Vc, dtype, S, seqlens, batch, Hq, Hkv, Lmax, d, B,
+                                      scale, O, idx, workspace,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ssa_status ssa_device_error(int* code) {
+  if (code == nullptr) return SSA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SSA_ERR_CUDA;
+  int a = ssa::read_and_reset_attn_tc_error();
+  int b = ssa::read_and_reset_decode_error();
+  *code = a != 0 ? a : b;
+  return SSA_OK;
+}
+
+}  // extern "C"

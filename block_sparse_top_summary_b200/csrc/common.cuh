@@ -1,0 +1,175 @@
+// Device helpers shared by the kernels of the block-sparse attention library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssa.h"
+
+namespace ssa {
+
+constexpr int kWarp = 32;
+
+// Elements of T in one 16-byte vector load.
+template <typename T>
+struct Vec16 {
+  static constexpr int n = 16 / sizeof(T);
+};
+
+// Unpack one 16-byte chunk into floats (exact for fp32 and bf16).
+__device__ __forceinline__ void unpack16(const uint4& v, float* out, const float*) {
+  out[0] = __uint_as_float(v.x);
+  out[1] = __uint_as_float(v.y);
+  out[2] = __uint_as_float(v.z);
+  out[3] = __uint_as_float(v.w);
+}
+
+__device__ __forceinline__ void bf16x2_to_f(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+
+__device__ __forceinline__ void unpack16(const uint4& v, float* out, const __nv_bfloat16*) {
+  bf16x2_to_f(v.x, out[0], out[1]);
+  bf16x2_to_f(v.y, out[2], out[3]);
+  bf16x2_to_f(v.z, out[4], out[5]);
+  bf16x2_to_f(v.w, out[6], out[7]);
+}
+
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Streaming 16-byte load that does not allocate in L1.
+__device__ __forceinline__ uint4 ldg16_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void store_out(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_out(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+// Order-preserving map from fp32 to uint32: a > b (as floats, no NaN) iff key(a) > key(b).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Top-k selection by one warp over n candidate scores held in shared memory.
+//
+// Candidate e (0 <= e < n) is block index first + e.  The k highest scores
+// are kept, equal scores going to the lower index; the chosen block indices
+// are written to out[0 ..) in ascending order and their number returned.
+// hist: 256 words of shared memory private to this warp.
+// The k-th largest key is found by a 4-pass MSB-first radix select (8 bits
+// per pass); the compaction pass then walks the candidates in index order and
+// takes every key above the threshold plus the first `need` keys equal to it.
+__device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, int first,
+                                                int32_t* out, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  if (k <= 0 || n <= 0) return 0;
+  if (k >= n) {
+    for (int e = lane; e < n; e += 32) out[e] = first + e;
+    return n;
+  }
+  uint32_t prefix = 0, pmask = 0;
+  int need = k;  // how many of the keys matching `prefix` are still to be taken
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int base = 0; base < n; base += 32) {
+      const int e = base + lane;
+      const bool ok = e < n;
+      const uint32_t key = ok ? order_key(sc[e]) : 0u;
+      const bool hit = ok && ((key & pmask) == prefix);
+      const uint32_t digit = (key >> shift) & 255u;
+      const uint32_t act = __ballot_sync(0xffffffffu, hit);
+      if (hit) {
+        const uint32_t peers = __match_any_sync(act, digit);
+        if ((peers & lanemask_lt()) == 0) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+      }
+    }
+    __syncwarp();
+    // Find the digit dd with  sum_{b > dd} hist[b] < need <= sum_{b >= dd} hist[b].
+    // Lane L owns bins 255-8L-7 .. 255-8L (descending), scanned high to low.
+    uint32_t c[8];
+    uint32_t local = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      c[q] = hist[255 - (lane * 8 + q)];
+      local += c[q];
+    }
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - local;  // count in bins above this lane's range
+    const bool mine = (excl < (uint32_t)need) && ((uint32_t)need <= incl);
+    const uint32_t who = __ballot_sync(0xffffffffu, mine);
+    const int src = __ffs(who) - 1;
+    uint32_t dd = 0, above = 0;
+    if (lane == src) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (run + c[q] >= (uint32_t)need) {
+          dd = 255u - (uint32_t)(lane * 8 + q);
+          above = run;
+          break;
+        }
+        run += c[q];
+      }
+    }
+    dd = __shfl_sync(0xffffffffu, dd, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    prefix |= dd << shift;
+    pmask |= 255u << shift;
+    need -= (int)above;
+    __syncwarp();
+  }
+  // prefix is now the k-th largest key; take all keys > prefix and the first
+  // `need` keys == prefix in ascending index order.
+  int pos = 0, eq_seen = 0;
+  for (int base = 0; base < n; base += 32) {
+    const int e = base + lane;
+    const bool ok = e < n;
+    const uint32_t key = ok ? order_key(sc[e]) : 0u;
+    const bool gt = ok && key > prefix;
+    const bool eq = ok && key == prefix;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const int eq_rank = eq_seen + __popc(eqm & lanemask_lt());
+    const bool take = gt || (eq && eq_rank < need);
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[pos + __popc(tm & lanemask_lt())] = first + e;
+    pos += __popc(tm);
+    eq_seen += __popc(eqm);
+  }
+  return pos;
+}
+
+}  // namespace ssa

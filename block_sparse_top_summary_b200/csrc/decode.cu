@@ -1,0 +1,443 @@
+// One decode step of block-sparse attention with top-k summary routing
+// (DashAttention page, "Contribuições Principais" 4, incremental decoding;
+// The Sparse Frontier page, RQ2: decode keeps the whole KV cache and loads
+// only the selected blocks, so its cost is memory traffic).
+//
+// Two launches, both HBM-bound:
+//   1. route: one CTA per (sequence, KV head).  The group-mean query scores
+//      the summaries of the complete blocks 1 .. last-1 (each warp takes 32
+//      summaries per step; lane l holds d/32 coordinates; a 31-shuffle
+//      butterfly leaves dot product l in lane l), then one warp runs the exact
+//      radix top-k (ties to the lower index).  The block list goes to the
+//      scratch area (and to the caller's idx if given).
+//   2. split-KV attention: one CTA per (split, sequence, KV head).  Each split
+//      owns a contiguous run of the selected blocks; every block's K rows and
+//      V rows are contiguous in the BHND cache, so each is fetched with ONE
+//      untiled bulk copy (TMA) into shared memory, all issued up front on one
+//      mbarrier.  The CTA computes the G heads' logits, a local softmax
+//      (max m, sum l, unnormalised o) and writes that partial; the last CTA of
+//      a (sequence, KV head) to finish (atomic counter) merges the partials
+//      with a log-sum-exp combine and writes O.
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace ssa {
+
+__device__ int g_decode_error = 0;
+
+namespace {
+
+constexpr int kMaxG = 8;            // query heads per KV head handled by the split kernel
+constexpr uint32_t kWaitLimit = 1u << 24;  // bounded mbarrier polls
+
+__device__ __forceinline__ float reduce32_transpose(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float send = upper ? v[k] : v[k + half];
+      const float keep = upper ? v[k + half] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- 1. route
+template <typename T, int D>
+__global__ void __launch_bounds__(256) decode_route_kernel(
+    const T* __restrict__ q, const float* __restrict__ S, const int32_t* __restrict__ seqlens,
+    int Hq, int Hkv, int Lmax, int B, int nsum, int kk, int width, int32_t* __restrict__ ws_idx,
+    int32_t* __restrict__ ws_cnt, int* __restrict__ ws_ctr, int32_t* __restrict__ idx_out,
+    float inv_sqrt_d) {
+  constexpr int SL = D / 32;
+  extern __shared__ __align__(16) float smem[];
+  float* qb = smem;                                          // [D]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(qb + D);      // [256]
+  float* sc = reinterpret_cast<float*>(hist + 256);          // [nsum]
+  const int bg = blockIdx.x;
+  const int b = bg / Hkv;
+  const int g = bg - b * Hkv;
+  const int G = Hq / Hkv;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int L = seqlens[b];
+  const bool valid = (L >= 1) && (L <= Lmax);
+  const int last = valid ? (L - 1) / B : 0;
+  const int n = valid ? max(last - 1, 0) : 0;  // candidates 1 .. last-1
+  if (t == 0) ws_ctr[bg] = 0;                   // reset the split counter for pass 2
+
+  if (t < D) {
+    float s = 0.f;
+    for (int h = 0; h < G; ++h) s += (float)q[((int64_t)b * Hq + g * G + h) * D + t];
+    qb[t] = s / (float)G;
+  }
+  __syncthreads();
+  {
+    float qs[SL];
+#pragma unroll
+    for (int e = 0; e < SL; ++e) qs[e] = qb[lane * SL + e];
+    const float* Sg = S + (int64_t)bg * nsum * D + lane * SL;
+    for (int j0 = 1 + warp * 32; j0 <= n; j0 += 32 * 8) {
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int j = min(j0 + c, n);
+        float a = 0.f;
+        if constexpr (SL == 4) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)j * D));
+          a = fmaf(x.x, qs[0], a);
+          a = fmaf(x.y, qs[1], a);
+          a = fmaf(x.z, qs[2], a);
+          a = fmaf(x.w, qs[3], a);
+        } else {
+          const float2 x = __ldg(reinterpret_cast<const float2*>(Sg + (int64_t)j * D));
+          a = fmaf(x.x, qs[0], a);
+          a = fmaf(x.y, qs[1], a);
+        }
+        v[c] = a;
+      }
+      const float dot = reduce32_transpose(v);
+      const int j = j0 + lane;
+      if (j <= n) sc[j - 1] = dot * inv_sqrt_d;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int32_t* row = ws_idx + (int64_t)bg * width;
+    int n_sel = 0;
+    if (valid) {
+      n_sel = 1;
+      if (last >= 1) {
+        const int m = warp_select_topk(sc, n, kk, 1, row + 1, hist);
+        __syncwarp();
+        if (lane == 0) row[m + 1] = last;
+        n_sel = m + 2;
+      }
+      if (lane == 0) row[0] = 0;
+    }
+    for (int p = n_sel + lane; p < width; p += 32) row[p] = -1;
+    if (lane == 0) ws_cnt[bg] = n_sel;
+    __syncwarp();
+    if (idx_out != nullptr) {
+      for (int p = lane; p < width; p += 32) idx_out[(int64_t)bg * width + p] = row[p];
+    }
+  }
+}
+
+// -------------------------------------------------------- 2. split-KV attention
+// Partial record per (sequence, KV head, split): m[G], l[G], o[G][D] (fp32,
+// log2 domain, o unnormalised).
+template <int D>
+__host__ __device__ constexpr int part_floats(int G) {
+  return G * (D + 2);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) decode_split_kernel(
+    const T* __restrict__ q, const T* __restrict__ Kc, const T* __restrict__ Vc,
+    const int32_t* __restrict__ seqlens, int Hq, int Hkv, int Lmax, int B, int width, int splits,
+    int per_split, const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
+    float* __restrict__ ws_part, int* __restrict__ ws_ctr, T* __restrict__ O,
+    float scale_log2) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const int G = Hq / Hkv;
+  const int split = blockIdx.x;
+  const int bg = blockIdx.y;
+  const int b = bg / Hkv;
+  const int g = bg - b * Hkv;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int nk_max = per_split * B;  // keys this CTA can hold
+
+  // shared layout: K rows | V rows | qs[G][D] | p[nk_max][G] | red | bar
+  T* Ks = reinterpret_cast<T*>(smem_raw);
+  T* Vs = Ks + (size_t)nk_max * D;
+  float* qs = reinterpret_cast<float*>(Vs + (size_t)nk_max * D);
+  float* ps = qs + kMaxG * D;                  // [nk_max][kMaxG], later [4][kMaxG][D]
+  const size_t ps_floats = max((size_t)nk_max * kMaxG, (size_t)(256 / (D / 2)) * kMaxG * D);
+  float* red = ps + ps_floats;                 // [8][kMaxG] + [kMaxG]
+  __shared__ uint64_t bar;
+  __shared__ int s_last;
+
+  const int L = seqlens[b];
+  const int ns = ws_cnt[bg];
+  const int s0 = split * per_split;
+  const int s1 = min(s0 + per_split, ns);
+  const int64_t kvbase = (int64_t)bg * Lmax;
+
+  // ---- issue every block's K and V bulk copies up front
+  int nkeys = 0;  // keys held, in selection order
+  if (s0 < s1) {
+    if (t == 0) {
+      ptx::mbar_init(&bar, 1);
+      ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (t == 0) {
+      uint32_t total = 0;
+      for (int s = s0; s < s1; ++s) {
+        const int j = ws_idx[(int64_t)bg * width + s];
+        total += 2u * (uint32_t)(min(B, L - j * B) * D * (int)sizeof(T));
+      }
+      ptx::mbar_arrive_expect_tx(&bar, total);
+      int off = 0;
+      for (int s = s0; s < s1; ++s) {
+        const int j = ws_idx[(int64_t)bg * width + s];
+        const int rows = min(B, L - j * B);
+        const uint32_t bytes = (uint32_t)(rows * D * (int)sizeof(T));
+        ptx::bulk_g2s(Ks + (size_t)off * D, Kc + (kvbase + (int64_t)j * B) * D, bytes, &bar);
+        ptx::bulk_g2s(Vs + (size_t)off * D, Vc + (kvbase + (int64_t)j * B) * D, bytes, &bar);
+        off += rows;
+      }
+    }
+    for (int s = s0; s < s1; ++s) {
+      const int j = ws_idx[(int64_t)bg * width + s];
+      nkeys += min(B, L - j * B);
+    }
+  }
+  // queries, pre-scaled into the log2 domain
+  for (int e = t; e < G * D; e += blockDim.x) {
+    const int h = e / D;
+    qs[h * D + (e - h * D)] = (float)q[((int64_t)b * Hq + g * G + h) * D + (e - h * D)] * scale_log2;
+  }
+  bool ok = true;
+  if (s0 < s1) ok = ptx::mbar_wait_bounded(&bar, 0, kWaitLimit);
+  if (!ok) atomicCAS(&g_decode_error, 0, (int)SSA_ERR_TIMEOUT);
+  __syncthreads();
+
+  float* part = ws_part + ((int64_t)bg * splits + split) * part_floats<D>(G);
+  // ---- logits: thread per key, rotated 16-byte chunks to spread smem banks
+  constexpr int EPC = Vec16<T>::n;
+  constexpr int CPR = D / EPC;
+  float mloc[kMaxG];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) mloc[h] = -INFINITY;
+  if (ok) {
+    for (int k = t; k < nkeys; k += blockDim.x) {
+      float acc[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
+      const T* kr = Ks + (size_t)k * D;
+      for (int c0 = 0; c0 < CPR; ++c0) {
+        const int c = (c0 + k) % CPR;
+        float f[EPC];
+        unpack16(*reinterpret_cast<const uint4*>(kr + c * EPC), f, (const T*)nullptr);
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+          if (h < G) {
+            const float* qh = qs + h * D + c * EPC;
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) acc[h] = fmaf(f[e], qh[e], acc[h]);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h < G) {
+          ps[k * kMaxG + h] = acc[h];
+          mloc[h] = fmaxf(mloc[h], acc[h]);
+        }
+      }
+    }
+  }
+  // CTA max per head
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) {
+    const float w = warp_max(mloc[h]);
+    if (lane == 0) red[warp * kMaxG + h] = w;
+  }
+  __syncthreads();
+  if (t < kMaxG) {
+    float mm = -INFINITY;
+    for (int w = 0; w < 8; ++w) mm = fmaxf(mm, red[w * kMaxG + t]);
+    red[8 * kMaxG + t] = mm;
+  }
+  __syncthreads();
+  // p = 2^(s - m), sums
+  float lloc[kMaxG];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) lloc[h] = 0.f;
+  for (int k = t; k < nkeys; k += blockDim.x) {
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < G) {
+        const float p = exp2f(ps[k * kMaxG + h] - red[8 * kMaxG + h]);
+        ps[k * kMaxG + h] = p;
+        lloc[h] += p;
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) {
+    const float w = warp_sum(lloc[h]);
+    if (lane == 0) red[warp * kMaxG + h] = w;
+  }
+  __syncthreads();
+  if (t < G) {
+    float ll = 0.f;
+    for (int w = 0; w < 8; ++w) ll += red[w * kMaxG + t];
+    part[t] = red[8 * kMaxG + t];  // m
+    part[G + t] = ll;              // l
+  }
+  // o[h][d] = sum_k p[k][h] V[k][d]: thread owns a pair of coordinates and a
+  // quarter of the keys; quarters meet in shared memory (reusing ps's tail).
+  {
+    const int dp = t % (D / 2);
+    const int kq = t / (D / 2);
+    const int nq4 = 256 / (D / 2);
+    float acc[kMaxG][2];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) acc[h][0] = acc[h][1] = 0.f;
+    for (int k = kq; k < nkeys; k += nq4) {
+      float v0, v1;
+      if constexpr (sizeof(T) == 2) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(Vs + (size_t)k * D + 2 * dp);
+        bf16x2_to_f(w, v0, v1);
+      } else {
+        const float2 w = *reinterpret_cast<const float2*>(Vs + (size_t)k * D + 2 * dp);
+        v0 = w.x;
+        v1 = w.y;
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) {
+        if (h < G) {
+          const float p = ps[k * kMaxG + h];
+          acc[h][0] = fmaf(p, v0, acc[h][0]);
+          acc[h][1] = fmaf(p, v1, acc[h][1]);
+        }
+      }
+    }
+    __syncthreads();  // everyone is done reading ps
+    float* ored = ps;  // [nq4][kMaxG][D]
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < G) {
+        ored[((size_t)kq * kMaxG + h) * D + 2 * dp] = acc[h][0];
+        ored[((size_t)kq * kMaxG + h) * D + 2 * dp + 1] = acc[h][1];
+      }
+    }
+    __syncthreads();
+    for (int e = t; e < G * D; e += blockDim.x) {
+      const int h = e / D, dd = e - h * D;
+      float s = 0.f;
+      for (int z = 0; z < nq4; ++z) s += ored[((size_t)z * kMaxG + h) * D + dd];
+      part[2 * G + h * D + dd] = s;
+    }
+  }
+  // ---- the last split of this (sequence, KV head) merges the partials
+  __threadfence();
+  __syncthreads();
+  if (t == 0) s_last = (atomicAdd(&ws_ctr[bg], 1) == splits - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* parts = ws_part + (int64_t)bg * splits * part_floats<D>(G);
+  for (int e = t; e < G * D; e += blockDim.x) {
+    const int h = e / D, dd = e - h * D;
+    T* op = O + ((int64_t)b * Hq + g * G + h) * D + dd;
+    if (ns == 0) {
+      store_out(op, 0.f);
+      continue;
+    }
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(parts + (int64_t)s * part_floats<D>(G) + h));
+    float num = 0.f, den = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float* ps_ = parts + (int64_t)s * part_floats<D>(G);
+      const float ms = __ldcg(ps_ + h);
+      if (ms == -INFINITY) continue;
+      const float w = exp2f(ms - M);
+      den = fmaf(w, __ldcg(ps_ + G + h), den);
+      num = fmaf(w, __ldcg(ps_ + 2 * G + h * D + dd), num);
+    }
+    store_out(op, num / den);
+  }
+}
+
+DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int Lmax) {
+  DecodePlan p{};
+  p.G = Hq / Hkv;
+  p.nblk_max = (Lmax + B - 1) / B;
+  p.kk = topk < p.nblk_max ? topk : p.nblk_max;
+  p.width = p.kk + 2;
+  // about 32 KB of K+V per split (two 16 KB blocks at B=64, d=128, bf16)
+  const int blk_bytes = 2 * B * d * 2;
+  p.per_split = blk_bytes >= 32768 ? 1 : 32768 / blk_bytes;
+  p.splits = (p.width + p.per_split - 1) / p.per_split;
+  const size_t bg = (size_t)batch * Hkv;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  p.off_idx = 0;
+  p.off_cnt = up(p.off_idx + bg * p.width * sizeof(int32_t));
+  p.off_ctr = up(p.off_cnt + bg * sizeof(int32_t));
+  p.off_part = up(p.off_ctr + bg * sizeof(int32_t));
+  p.bytes = up(p.off_part + bg * p.splits * (size_t)p.G * (d + 2) * sizeof(float));
+  return p;
+}
+
+template <typename T, int D>
+static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const void* Kc,
+                                   const void* Vc, const float* S, const int32_t* seqlens,
+                                   int batch, int Hq, int Hkv, int Lmax, int B, float scale,
+                                   void* O, int32_t* idx_out, void* ws, cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
+  int32_t* ws_idx = reinterpret_cast<int32_t*>(w + p.off_idx);
+  int32_t* ws_cnt = reinterpret_cast<int32_t*>(w + p.off_cnt);
+  int* ws_ctr = reinterpret_cast<int*>(w + p.off_ctr);
+  float* ws_part = reinterpret_cast<float*>(w + p.off_part);
+  const int nsum = Lmax / B;
+  const size_t smem1 = sizeof(float) * (D + 256 + (size_t)(nsum > 0 ? nsum : 1));
+  cudaError_t e = cudaFuncSetAttribute(decode_route_kernel<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  if (e != cudaSuccess) return e;
+  decode_route_kernel<T, D><<<batch * Hkv, 256, smem1, st>>>(
+      (const T*)q, S, seqlens, Hq, Hkv, Lmax, B, nsum, p.kk, p.width, ws_idx, ws_cnt, ws_ctr,
+      idx_out, 1.0f / sqrtf((float)D));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int nk_max = p.per_split * B;
+  const int nq4 = 256 / (D / 2);
+  size_t ps_floats = (size_t)nk_max * kMaxG;
+  const size_t ored_floats = (size_t)nq4 * kMaxG * D;
+  if (ored_floats > ps_floats) ps_floats = ored_floats;
+  const size_t smem2 = 2 * (size_t)nk_max * D * sizeof(T) +
+                       sizeof(float) * ((size_t)kMaxG * D + ps_floats + 9 * kMaxG);
+  e = cudaFuncSetAttribute(decode_split_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem2);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.splits, batch * Hkv);
+  decode_split_kernel<T, D><<<grid, 256, smem2, st>>>(
+      (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, p.splits,
+      p.per_split, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O, scale * 1.4426950408889634f);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
+                          ssa_dtype dt, const float* S, const int32_t* seqlens, int batch, int Hq,
+                          int Hkv, int Lmax, int d, int B, float scale, void* O, int32_t* idx_out,
+                          void* ws, cudaStream_t st) {
+  if (dt == SSA_BF16) {
+    return d == 128 ? launch_decode_t<__nv_bfloat16, 128>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv,
+                                                          Lmax, B, scale, O, idx_out, ws, st)
+                    : launch_decode_t<__nv_bfloat16, 64>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv,
+                                                         Lmax, B, scale, O, idx_out, ws, st);
+  }
+  return d == 128 ? launch_decode_t<float, 128>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv, Lmax, B,
+                                                scale, O, idx_out, ws, st)
+                  : launch_decode_t<float, 64>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv, Lmax, B,
+                                               scale, O, idx_out, ws, st);
+}
+
+int read_and_reset_decode_error() {
+  int v = 0;
+  cudaMemcpyFromSymbol(&v, g_decode_error, sizeof(int));
+  const int z = 0;
+  cudaMemcpyToSymbol(g_decode_error, &z, sizeof(int));
+  return v;
+}
+
+}  // namespace ssa

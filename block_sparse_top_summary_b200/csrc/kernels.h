@@ -1,0 +1,58 @@
+// Host-side launchers of the library's kernels (internal; the public ABI is ssa.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ssa.h"
+
+namespace ssa {
+
+cudaError_t launch_block_summary(const void* K, ssa_dtype dt, int batch, int Hkv, int N, int d,
+                                 int B, float* S, cudaStream_t st);
+
+// Largest number of query blocks ssa_route handles (its score rows live in
+// shared memory).
+constexpr int kRouteMaxBlocks = 4096;
+
+cudaError_t launch_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq, int Hkv,
+                         int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
+                         cudaStream_t st);
+
+// True when the tensor-core prefill kernel covers this shape.
+bool attn_tc_supported(ssa_dtype dt, int Hq, int Hkv, int d, int B);
+
+cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const int32_t* idx,
+                           const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
+                           int max_sel, float scale, void* O, float* lse, cudaStream_t st);
+
+cudaError_t launch_attn_simt(const void* Q, const void* K, const void* V, ssa_dtype dt,
+                             const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
+                             int N, int d, int B, int max_sel, float scale, void* O, float* lse,
+                             cudaStream_t st);
+
+// Decode: scratch layout and launch.
+struct DecodePlan {
+  int G;          // query heads per KV head
+  int nblk_max;   // ceil(Lmax / B)
+  int kk;         // effective top-k: min(topk, nblk_max)
+  int width;      // idx row width: kk + 2
+  int splits;     // CTAs per (sequence, KV head) in the split-KV pass
+  int per_split;  // selected blocks handled by one split CTA
+  size_t off_idx, off_cnt, off_part, off_ctr, bytes;
+};
+
+DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int Lmax);
+
+cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
+                          ssa_dtype dt, const float* S, const int32_t* seqlens, int batch, int Hq,
+                          int Hkv, int Lmax, int d, int B, float scale, void* O, int32_t* idx_out,
+                          void* ws, cudaStream_t st);
+
+// Device error words (one per translation unit that has bounded waits):
+// read and reset; returns the first non-zero code or 0.
+int read_and_reset_attn_tc_error();
+int read_and_reset_decode_error();
+
+}  // namespace ssa

@@ -1,0 +1,227 @@
+// Stage 1: routing.  Each query block scores the summaries of the complete
+// key blocks before it and keeps the top-k; sink block 0 and the diagonal are
+// always added (DashAttention page, "Estágio 1" and "Estágio 2", diagonal
+// branch; The Sparse Frontier page, RQ2, block-wise prefill selection; GSA
+// page, "Componentes Principais" 3).  Query heads of one GQA group share the
+// selection: their rows are pooled together (DashAttention page, "Estágio 1",
+// GQA handling).
+//
+// One fused kernel, one CTA of 256 threads per (tile of 8 query blocks,
+// batch x KV head):
+//   1. pool: stream the tile's Q rows (G heads x B rows x d per query block)
+//      with coalesced 16-byte loads into 8 fp32 means qbar (HBM-bound part);
+//   2. score: every warp takes 4 candidate summaries at a time; lane l holds
+//      d/32 coordinates of each summary and of the 8 qbar rows, so one
+//      coalesced load feeds 8*d/32 FMAs; the 32 partial dot products of a
+//      warp step are reduced with a 31-shuffle butterfly that leaves dot
+//      product l in lane l; scores land in shared memory;
+//   3. select: warp w selects for query block w of the tile with an exact
+//      4-pass radix select (ties to the lower index) and writes the ascending
+//      block list.
+// Tiles are dispatched heaviest first (late query blocks have the most
+// candidates).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ssa {
+
+namespace {
+
+constexpr int TQ = 8;  // query blocks per CTA (= warps per CTA)
+
+// Butterfly reduction of 32 per-lane values: afterwards lane l's v[0] holds
+// the warp-wide sum of value index l.
+__device__ __forceinline__ float reduce32_transpose(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float send = upper ? v[k] : v[k + half];
+      const float keep = upper ? v[k + half] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
+}  // namespace
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
+                                                    const float* __restrict__ S,
+                                                    int32_t* __restrict__ idx,
+                                                    int32_t* __restrict__ cnt, int Hq, int Hkv,
+                                                    int N, int B, int nq, int nfull, int topk,
+                                                    int max_sel, int ntiles, int sc_stride,
+                                                    float inv_sqrt_d) {
+  constexpr int EPC = Vec16<T>::n;
+  constexpr int CPR = D / EPC;
+  constexpr int RL = 256 / CPR;
+  constexpr int SL = D / 32;  // summary coordinates per lane
+  extern __shared__ __align__(16) float smem[];
+  float* qbar = smem;                                        // [TQ][D]
+  float* red = qbar + TQ * D;                                // [RL][D]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(red + RL * D);  // [TQ][256]
+  float* sc = reinterpret_cast<float*>(hist + TQ * 256);     // [TQ][sc_stride]
+
+  const int t = threadIdx.x;
+  const int lane = t & 31;
+  const int warp = t >> 5;
+  const int bg = blockIdx.x;  // b * Hkv + g
+  const int tile = ntiles - 1 - (int)blockIdx.y;
+  const int G = Hq / Hkv;
+  const int b = bg / Hkv;
+  const int g = bg - b * Hkv;
+  const int i0 = tile * TQ;
+  const int i1 = min(i0 + TQ, nq);
+
+  // ---- 1. pool Q over (rows of the block) x (heads of the group)
+  {
+    const int cc = t % CPR;
+    const int rl = t / CPR;
+    for (int qi = i0; qi < i1; ++qi) {
+      const int rows = min(B, N - qi * B);
+      const int R = G * rows;
+      float acc[EPC];
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+      const T* blk = Q + ((int64_t)(b * Hq + g * G) * N + (int64_t)qi * B) * D + cc * EPC;
+      int rr = rl;
+      for (; rr + 3 * RL < R; rr += 4 * RL) {
+        uint4 v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int r = rr + q * RL;
+          const int h = r / rows;
+          v[q] = ldg16_stream(blk + ((int64_t)h * N + (r - h * rows)) * D);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float f[EPC];
+          unpack16(v[q], f, (const T*)nullptr);
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+        }
+      }
+      for (; rr < R; rr += RL) {
+        const int h = rr / rows;
+        float f[EPC];
+        unpack16(ldg16_stream(blk + ((int64_t)h * N + (rr - h * rows)) * D), f, (const T*)nullptr);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+      }
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) red[rl * D + cc * EPC + e] = acc[e];
+      __syncthreads();
+      if (t < D) {
+        float s = 0.f;
+        for (int q = 0; q < RL; ++q) s += red[q * D + t];
+        qbar[(qi - i0) * D + t] = s / (float)R;
+      }
+      __syncthreads();
+    }
+  }
+
+  // ---- 2. scores for candidates j = 1 .. i1-2 against all TQ rows
+  const int ncand = max(i1 - 2, 0);
+  {
+    float qs[TQ][SL];
+#pragma unroll
+    for (int q = 0; q < TQ; ++q)
+#pragma unroll
+      for (int e = 0; e < SL; ++e) qs[q][e] = qbar[q * D + lane * SL + e];
+    const float* Sg = S + (int64_t)bg * nfull * D + lane * SL;
+    for (int j0 = 1 + warp * 4; j0 <= ncand; j0 += 4 * (256 / 32)) {
+      float sv[4][SL];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = min(j0 + c, ncand);
+        if (SL == 4) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)j * D));
+          sv[c][0] = x.x; sv[c][1] = x.y; sv[c][2 % SL] = x.z; sv[c][3 % SL] = x.w;
+        } else {
+          const float2 x = __ldg(reinterpret_cast<const float2*>(Sg + (int64_t)j * D));
+          sv[c][0] = x.x; sv[c][1 % SL] = x.y;
+        }
+      }
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int q = 0; q < TQ; ++q) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < SL; ++e) a = fmaf(sv[c][e], qs[q][e], a);
+          v[c * TQ + q] = a;
+        }
+      const float dot = reduce32_transpose(v);
+      const int c = lane / TQ;
+      const int q = lane % TQ;
+      const int j = j0 + c;
+      if (j <= ncand) sc[q * sc_stride + (j - 1)] = dot * inv_sqrt_d;
+    }
+  }
+  __syncthreads();
+
+  // ---- 3. per query block: top-k, then {0} U R U {i} ascending, -1 padded
+  {
+    const int i = i0 + warp;
+    if (i < i1) {
+      int32_t* row = idx + ((int64_t)bg * nq + i) * max_sel;
+      int n_sel = 1;  // block 0
+      if (i >= 1) {
+        const int m = warp_select_topk(sc + warp * sc_stride, i - 1, topk, 1, row + 1,
+                                       hist + warp * 256);
+        n_sel = m + 2;
+        __syncwarp();
+        if (lane == 0) row[m + 1] = i;
+      }
+      if (lane == 0) {
+        row[0] = 0;
+        cnt[(int64_t)bg * nq + i] = n_sel;
+      }
+      for (int p = n_sel + lane; p < max_sel; p += 32) row[p] = -1;
+    }
+  }
+}
+
+template <typename T, int D>
+static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int Hq, int Hkv, int N,
+                                  int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
+                                  cudaStream_t st) {
+  constexpr int EPC = Vec16<T>::n;
+  constexpr int RL = 256 / (D / EPC);
+  const int nq = (N + B - 1) / B;
+  const int nfull = N / B;
+  const int ntiles = (nq + TQ - 1) / TQ;
+  const int sc_stride = nq > 2 ? nq - 2 : 1;
+  const size_t smem = sizeof(float) * ((size_t)TQ * D + (size_t)RL * D + (size_t)TQ * 256 +
+                                       (size_t)TQ * sc_stride);
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(batch * Hkv, ntiles);
+  route_kernel<T, D><<<grid, 256, smem, st>>>((const T*)Q, S, idx, cnt, Hq, Hkv, N, B, nq, nfull,
+                                              topk, max_sel, ntiles, sc_stride,
+                                              1.0f / sqrtf((float)D));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq, int Hkv,
+                         int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
+                         cudaStream_t st) {
+  if (dt == SSA_BF16) {
+    return d == 128 ? launch_route_t<__nv_bfloat16, 128>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel,
+                                                         idx, cnt, st)
+                    : launch_route_t<__nv_bfloat16, 64>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel,
+                                                        idx, cnt, st);
+  }
+  return d == 128 ? launch_route_t<float, 128>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt,
+                                               st)
+                  : launch_route_t<float, 64>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt,
+                                              st);
+}
+
+}  // namespace ssa

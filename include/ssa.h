@@ -1,0 +1,176 @@
+/*
+ * ssa.h - C ABI of the block-sparse attention library with top-k summary routing.
+ *
+ * The method (DashAttention page, "Metodologia", stages 0-2; GSA page,
+ * "Componentes Principais" 2-3; SSA page, "2. Metodologia", sparse stream):
+ * keys are cut into contiguous blocks of B rows and each block is summarised
+ * by its mean key; each query block scores the summaries of the complete key
+ * blocks before it and keeps the top-k; the sink block 0 and the causal
+ * diagonal block are always added; exact softmax attention then runs over the
+ * keys of the selected blocks only.  Decode runs the same stages for one
+ * query token per sequence against a KV cache.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Layout BHND: Q is [batch, Hq, N, d], K and V are [batch, Hkv, N, d], all
+ *   contiguous with d innermost.  Query head h uses KV head h / (Hq / Hkv)
+ *   (grouped-query attention, GQA).
+ * - Every pointer argument is a DEVICE pointer, 16-byte aligned, owned by the
+ *   caller.  The library allocates and frees nothing and keeps no state between
+ *   calls other than a device-side error word (see ssa_device_error).
+ * - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and nothing synchronises with the host.
+ * - Argument checks run on the host before any launch; a failed check returns
+ *   an error code and launches nothing.  A launch failure returns SSA_ERR_CUDA.
+ * - Supported: d in {64, 128}; B a multiple of 16 in [16, 128]; Hq % Hkv == 0;
+ *   dtype SSA_F32 or SSA_BF16 (all of Q, K, V, O share it).
+ * - Block counts: nq = ceil(N / B) query blocks; nfull = floor(N / B) complete
+ *   key blocks.  A trailing partial block has no summary and is only ever
+ *   attended as a diagonal block.
+ */
+#ifndef SSA_H
+#define SSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSA_OK = 0,
+  SSA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer */
+  SSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (d, B, dtype, sizes) */
+  SSA_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+  SSA_ERR_TIMEOUT = 4      /* a bounded device-side wait expired (see ssa_device_error) */
+} ssa_status;
+
+typedef enum { SSA_F32 = 0, SSA_BF16 = 1 } ssa_dtype;
+
+/* Opaque CUDA stream handle; binary-compatible with cudaStream_t. */
+typedef struct CUstream_st* ssa_stream;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* ssa_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int ssa_version(void);
+
+/*
+ * Stage 0, block summary (DashAttention page, "Estágio 0": with the learned
+ * summary query at zero the block summary is the uniform mean; GSA page,
+ * "Componentes Principais" 2: MoBA's mean pooling).
+ *
+ *   S[b, g, j, :] = (1 / B) * sum_{t = jB}^{jB + B - 1} K[b, g, t, :]   for j < nfull
+ *
+ * K: [batch, Hkv, N, d] of `dtype`.  S: [batch, Hkv, nfull, d] fp32 (written).
+ * N < B is valid and writes nothing.
+ */
+ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv, int N, int d,
+                             int B, float* S, ssa_stream stream);
+
+/*
+ * Stage 1, routing (DashAttention page, "Estágio 1": each query scores the
+ * block summaries; GQA heads sharing a KV head share one support; The Sparse
+ * Frontier page, RQ2: block-wise selection in prefill; GSA page,
+ * "Componentes Principais" 3: top-k of the blocks).
+ *
+ * For every (b, KV head g, query block i):
+ *   qbar = mean of Q over the rows of block i and the heads of group g;
+ *   s_j  = qbar . S[b, g, j, :] / sqrt(d) for candidates j = 1 .. i-1;
+ *   R    = the min(topk, i-1) candidates of highest s_j, equal scores going to
+ *          the lower block index;
+ *   selection = {0} U R U {i}, written ascending.
+ * Scores are computed in fp32 from the fp32 summaries.
+ *
+ * Q: [batch, Hq, N, d] of `dtype`.  S: [batch, Hkv, nfull, d] fp32.
+ * idx: [batch, Hkv, nq, max_sel] int32 (written; entries past cnt are -1).
+ * cnt: [batch, Hkv, nq] int32 (written).
+ * topk >= 0; any topk >= nq selects every candidate.
+ * max_sel must be >= min(topk, max(nq - 2, 0)) + 2.
+ * SSA_ERR_UNSUPPORTED if nq > 4096 (the score rows of a tile of query blocks
+ * are held in shared memory).
+ */
+ssa_status ssa_route(const void* Q, ssa_dtype dtype, const float* S, int batch, int Hq, int Hkv,
+                     int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
+                     ssa_stream stream);
+
+/*
+ * Stage 2, exact softmax attention over the selected blocks (SSA page,
+ * "2. Metodologia", sparse stream; DashAttention page, "Estágio 2", attention
+ * restricted to the routed blocks plus the diagonal branch).
+ *
+ * For query row t of head h (block i = t / B, group g = h / (Hq / Hkv)) the
+ * keys are the rows of the blocks idx[b, g, i, 0 .. cnt-1] at key positions
+ * <= t (the causal mask binds only on the diagonal block):
+ *   O[b, h, t, :] = softmax(scale * q_t . K_sel^T) V_sel
+ *   lse[b, h, t]  = log(sum exp(scale * q_t . K_sel^T))   (natural log)
+ * Accumulation is fp32; O is rounded to `dtype` (round to nearest even).
+ *
+ * idx/cnt as written by ssa_route (entries ascending, each in [0, i], the
+ * diagonal i included).  lse may be NULL.  scale > 0 (normally 1/sqrt(d)).
+ * bf16 with d = 128, B in {64, 128} and (Hq/Hkv)*B a multiple of 256 runs on
+ * the tensor cores (TMA + tcgen05 + TMEM); every other shape runs a SIMT kernel.
+ * A bounded device-side wait that expires sets the device error word
+ * (SSA_ERR_TIMEOUT, see ssa_device_error) instead of hanging.
+ */
+ssa_status ssa_sparse_attn_fwd(const void* Q, const void* K, const void* V, ssa_dtype dtype,
+                               const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
+                               int N, int d, int B, int max_sel, float scale, void* O, float* lse,
+                               ssa_stream stream);
+
+/*
+ * 1 if ssa_sparse_attn_fwd runs this shape on the tensor cores, else 0 (the
+ * SIMT kernel).  Pure host query.
+ */
+int ssa_sparse_attn_uses_tensor_cores(ssa_dtype dtype, int Hq, int Hkv, int d, int B);
+
+/*
+ * Scratch size, in bytes, that ssa_decode needs for these sizes.
+ */
+ssa_status ssa_decode_workspace_size(int batch, int Hq, int Hkv, int Lmax, int d, int B,
+                                     int topk, size_t* bytes);
+
+/*
+ * One decode step (DashAttention page, "Contribuições Principais" 4:
+ * incremental decoding with the same stages; The Sparse Frontier page, RQ2:
+ * decode keeps the whole KV cache and loads only the selected blocks).
+ *
+ * Sequence b holds L = seqlens[b] tokens in its cache, the current token
+ * included, so the query sits at position L-1 and its diagonal block is
+ * last = (L-1) / B (possibly partial; its keys at positions >= L are masked).
+ *   qbar = mean over the group's heads of q;  s_j = qbar . S[b, g, j] / sqrt(d)
+ *   for the complete blocks j = 1 .. last-1; selection = {0} U top-k U {last}.
+ * The selected blocks are split across CTAs (split-KV) and the partial
+ * results are merged with a log-sum-exp combine.
+ *
+ * q: [batch, Hq, d]; Kc, Vc: [batch, Hkv, Lmax, d] of `dtype`;
+ * S: [batch, Hkv, Lmax / B, d] fp32 block summaries of the cache (only the
+ *    complete blocks before `last` are read);
+ * seqlens: [batch] int32, 1 <= seqlens[b] <= Lmax (read on the device; a value
+ *    out of range makes that sequence write zeros);
+ * O: [batch, Hq, d] of `dtype` (written);
+ * idx: NULL or [batch, Hkv, min(topk, ceil(Lmax / B)) + 2] int32 (written,
+ *    ascending, -1 padded);
+ * workspace: >= ssa_decode_workspace_size(...) bytes of device memory, 256-byte
+ *    aligned, contents on entry ignored.  Calls that share a workspace must
+ *    not overlap on the device.
+ */
+ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype dtype,
+                      const float* S, const int32_t* seqlens, int batch, int Hq, int Hkv, int Lmax,
+                      int d, int B, int topk, float scale, void* O, int32_t* idx, void* workspace,
+                      size_t ws_bytes, ssa_stream stream);
+
+/*
+ * Device error word: 0, or the ssa_status of the first bounded device-side
+ * wait that expired since the last reset.  Synchronises the device, then
+ * writes the word to *code and resets it to 0.
+ */
+ssa_status ssa_device_error(int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H */

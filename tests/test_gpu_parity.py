@@ -1,0 +1,243 @@
+"""GPU-vs-oracle parity on small inputs (several tiles, ragged tails, edge cases).
+
+Every GPU call goes through the C ABI (ctypes binding).  Selections must match
+the oracle exactly except near-ties (fp64 score gap < 1e-4 relative), which
+are counted; outputs are compared with the oracle recomputed on the GPU's own
+selection, at max-abs 1e-5 (fp32) or max-abs 2e-2 and relative-L2 5e-3 (bf16).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from parity import BF16_MAX_ABS, BF16_REL_L2, F32_MAX_ABS, compare_selection, out_errors
+from workloads import CONFIGS, planted_decode, planted_prefill, to_f64
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def ssa():
+    import block_sparse_top_summary_b200 as m
+    m.load_library()
+    return m
+
+
+def _check_out(gpu, ref, dtype):
+    ma, rel = out_errors(gpu, ref)
+    if dtype == "f32":
+        assert ma <= F32_MAX_ABS, (ma, rel)
+    else:
+        assert ma <= BF16_MAX_ABS and rel <= BF16_REL_L2, (ma, rel)
+    return ma, rel
+
+
+# ------------------------------------------------------------------ summary
+@pytest.mark.parametrize("batch,Hkv,N,d,B,dtype", [
+    (1, 1, 1024, 64, 64, "f32"),
+    (2, 3, 64 * 7 + 13, 128, 64, "bf16"),
+    (1, 2, 512, 128, 128, "f32"),
+    (1, 1, 300, 64, 16, "bf16"),
+    (2, 2, 4096, 128, 32, "bf16"),
+])
+def test_summary_parity(ssa, batch, Hkv, N, d, B, dtype):
+    _, K, _ = planted_prefill(batch, Hkv, Hkv, N, d, B, clusters=3, seed=1, dtype=dtype)
+    S = ssa.ssa_block_summary(K.to(DEV), B)
+    ref = O.block_summary(to_f64(K), B)
+    assert S.shape == ref.shape
+    ma, _ = out_errors(to_f64(S), ref)
+    assert ma <= 1e-5
+
+
+def test_summary_constant_blocks_exact(ssa):
+    c = torch.randint(-8, 8, (1, 2, 6, 128)).float()
+    K = c.repeat_interleave(64, dim=2).to(torch.bfloat16).contiguous()
+    S = ssa.ssa_block_summary(K.to(DEV), 64)
+    assert torch.equal(S.cpu(), c)
+
+
+# ------------------------------------------------------------------ routing
+def _route_case(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters, seed):
+    Q, K, _ = planted_prefill(batch, Hq, Hkv, N, d, B, clusters, seed=seed, dtype=dtype)
+    S = ssa.ssa_block_summary(K.to(DEV), B)
+    idx, cnt = ssa.ssa_route(Q.to(DEV), S, B, topk, Hkv)
+    Qf, Kf = to_f64(Q), to_f64(K)
+    oidx, ocnt, osc = O.route(Qf, O.block_summary(Kf, B), B, topk, Hkv)
+    return idx.cpu().numpy(), cnt.cpu().numpy(), oidx, ocnt, osc
+
+
+@pytest.mark.parametrize("batch,Hq,Hkv,N,d,B,topk,dtype,clusters", [
+    (1, 2, 1, 1024, 64, 64, 4, "f32", 0),            # the tiny workload
+    (1, 8, 2, 64 * 70 + 9, 128, 64, 6, "bf16", 5),   # ragged tail, 9 tiles of 8
+    (2, 4, 4, 2048, 64, 32, 0, "f32", 4),            # top-k = 0: sink + diagonal only
+    (1, 4, 1, 128 * 20, 128, 128, 1 << 30, "bf16", 3),  # "all"
+    (1, 16, 4, 128 * 33, 128, 128, 8, "bf16", 8),    # B = 128
+    (1, 4, 2, 16 * 300, 64, 16, 24, "bf16", 6),      # B = 16, many blocks
+])
+def test_route_parity(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters):
+    gi, gc, oi, oc, osc = _route_case(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters, 2)
+    assert np.array_equal(gc, oc)
+    w = oi.shape[-1]
+    assert np.all(gi[..., w:] == -1)
+    rows, near, bad = compare_selection(gi, gc, oi, oc,
+                                        lambda r: {j: osc[r][j] for j in range(osc.shape[-1])})
+    assert not bad, bad[:3]
+    assert near <= max(1, rows // 50)
+
+
+def test_route_tiny_matches_golden(ssa):
+    import json
+    import os
+    doc = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "tiny_oracle.json")))
+    c = CONFIGS["tiny"]
+    Q, K, _ = planted_prefill(c.batch, c.Hq, c.Hkv, c.N, c.d, c.B, c.clusters, c.seed, c.dtype)
+    S = ssa.ssa_block_summary(K.to(DEV), c.B)
+    idx, cnt = ssa.ssa_route(Q.to(DEV), S, c.B, c.topk, c.Hkv)
+    assert cnt[0, 0].tolist() == doc["cnt"]
+    assert idx[0, 0].tolist() == doc["idx"]
+
+
+def test_route_exact_ties_go_to_lower_index(ssa):
+    torch.manual_seed(0)
+    B, d, nb = 64, 128, 12
+    K = torch.randn(1, 1, nb * B, d) * 0.1
+    u = torch.randn(d)
+    blk = torch.randn(B, d) * 0.1 + u
+    for j in (2, 5, 7, 10):
+        K[0, 0, j * B:(j + 1) * B] = blk
+    Q = u.expand(1, 4, nb * B, d).contiguous()
+    S = ssa.ssa_block_summary(K.to(DEV), B)
+    idx, cnt = ssa.ssa_route(Q.to(DEV), S, B, 2, 1)
+    idx = idx.cpu()
+    assert idx[0, 0, 11, :cnt[0, 0, 11]].tolist() == [0, 2, 5, 11]
+    assert idx[0, 0, 8, :cnt[0, 0, 8]].tolist() == [0, 2, 5, 8]
+
+
+# ---------------------------------------------------------------- attention
+def _attn_case(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters, seed=3):
+    Q, K, V = planted_prefill(batch, Hq, Hkv, N, d, B, clusters, seed=seed, dtype=dtype)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    out, lse, idx, cnt, _ = ssa.prefill(Qd, Kd, Vd, B, topk)
+    ref, rlse = O.sparse_attention(to_f64(Q), to_f64(K), to_f64(V), idx.cpu().numpy(),
+                                   cnt.cpu().numpy(), B)
+    return out, lse, ref, rlse
+
+
+@pytest.mark.parametrize("batch,Hq,Hkv,N,d,B,topk,dtype,clusters", [
+    (1, 2, 1, 1024, 64, 64, 4, "f32", 0),             # the tiny workload
+    (1, 4, 2, 64 * 9 + 17, 128, 64, 3, "f32", 2),     # ragged, fp32 d=128
+    (2, 8, 2, 64 * 12 + 5, 128, 64, 4, "bf16", 4),    # bf16, G = 4, ragged
+    (1, 8, 2, 128 * 9, 128, 128, 3, "bf16", 3),       # bf16, B = 128
+    (1, 4, 4, 32 * 20 + 31, 64, 32, 5, "bf16", 3),    # G = 1, B = 32, d = 64
+    (1, 8, 1, 64 * 10, 128, 64, 1 << 30, "bf16", 0),  # all blocks (dense), G = 8
+])
+def test_attention_parity(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters):
+    out, lse, ref, rlse = _attn_case(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters)
+    _check_out(to_f64(out), ref, dtype)
+    np.testing.assert_allclose(to_f64(lse), rlse, rtol=0, atol=1e-4)
+
+
+def test_all_blocks_equals_dense_causal(ssa):
+    Q, K, V = planted_prefill(1, 8, 2, 64 * 16, 128, 64, 0, seed=5, dtype="bf16")
+    out, _, _, cnt, _ = ssa.prefill(Q.to(DEV), K.to(DEV), V.to(DEV), 64, 1 << 30)
+    assert cnt.cpu()[0, 0].tolist() == [i + 1 for i in range(16)]
+    q = to_f64(Q)
+    k = torch.from_numpy(to_f64(K)).repeat_interleave(4, 1)
+    v = torch.from_numpy(to_f64(V)).repeat_interleave(4, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q), k, v,
+                                                           is_causal=True).numpy()
+    _check_out(to_f64(out), ref, "bf16")
+
+
+def test_values_one_give_output_one(ssa):
+    for dtype, tol in (("f32", 1e-6), ("bf16", 1e-2)):
+        Q, K, V = planted_prefill(1, 8, 2, 64 * 8 + 3, 128, 64, 2, seed=6, dtype=dtype)
+        V = torch.ones_like(V)
+        out, _, _, _, _ = ssa.prefill(Q.to(DEV), K.to(DEV), V.to(DEV), 64, 2)
+        assert torch.max(torch.abs(out.float() - 1.0)).item() <= tol
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_poisoned_unselected_and_future_keys_do_not_change_output(ssa, dtype):
+    B, N, d = 64, 64 * 10, 128
+    Q, K, V = planted_prefill(1, 8, 2, N, d, B, 3, seed=7, dtype=dtype)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    i, t = 7, 7 * 64 + 20  # query block 7, check rows up to t
+    nq = N // B
+    idx = torch.full((1, 2, nq, 4), -1, dtype=torch.int32)
+    cnt = torch.ones(1, 2, nq, dtype=torch.int32)
+    idx[..., 0] = 0
+    idx[0, :, i, :3] = torch.tensor([0, 3, i], dtype=torch.int32)
+    cnt[0, :, i] = 3
+    idx, cnt = idx.to(DEV), cnt.to(DEV)
+    base, _ = ssa.ssa_sparse_attn_fwd(Qd, Kd, Vd, idx, cnt, B)
+    Kp, Vp = Kd.clone(), Vd.clone()
+    for j in range(nq):
+        if j not in (0, 3, i):
+            Kp[:, :, j * B:(j + 1) * B] = float("nan")
+            Vp[:, :, j * B:(j + 1) * B] = float("nan")
+    Kp[:, :, t + 1:(i + 1) * B] = 1e30
+    Vp[:, :, t + 1:(i + 1) * B] = -1e30
+    pois, _ = ssa.ssa_sparse_attn_fwd(Qd, Kp, Vp, idx, cnt, B)
+    rows = slice(i * B, t + 1)
+    assert torch.equal(base[:, :, rows], pois[:, :, rows])
+
+
+# ------------------------------------------------------------------ decode
+@pytest.mark.parametrize("batch,Hq,Hkv,Lmax,d,B,topk,dtype,seqlens", [
+    (3, 8, 2, 1000, 128, 64, 4, "bf16", [1000, 37, 64 * 5 + 1]),
+    (2, 4, 1, 64 * 40, 64, 64, 6, "f32", [64 * 40, 64 * 23 + 63]),
+    (4, 16, 4, 128 * 30, 128, 128, 5, "bf16", [128 * 30, 1, 128, 129]),
+    (2, 8, 1, 64 * 50, 128, 64, 1 << 30, "bf16", [64 * 50, 64 * 7 + 3]),   # all blocks
+    (2, 6, 2, 16 * 200, 64, 16, 12, "bf16", [16 * 200, 16 * 77 + 5]),      # G = 3, B = 16
+])
+def test_decode_parity(ssa, batch, Hq, Hkv, Lmax, d, B, topk, dtype, seqlens):
+    q, Kc, Vc, L = planted_decode(batch, Hq, Hkv, Lmax, d, B, clusters=5, seed=8, dtype=dtype,
+                                  seqlens=seqlens)
+    qd, Kd, Vd, Ld = q.to(DEV), Kc.to(DEV), Vc.to(DEV), L.to(DEV)
+    S = ssa.ssa_block_summary(Kd, B)
+    out, idx = ssa.ssa_decode(qd, Kd, Vd, S, Ld, B, topk)
+    gi = idx.cpu().numpy()
+    qf, Kf, Vf = to_f64(q), to_f64(Kc), to_f64(Vc)
+    Sf = np.stack([O.block_summary(Kf[b:b + 1], B)[0] for b in range(batch)])
+    oi, oc, osc = O.decode_route(qf, Sf, L.numpy(), B, topk)
+    gc = (gi >= 0).sum(-1)
+    rows, near, bad = compare_selection(gi, gc, oi, oc,
+                                        lambda r: {j: osc[r][j] for j in range(osc.shape[-1])})
+    assert not bad, bad[:3]
+    ref, _, _, _ = O.decode(qf, Kf, Vf, L.numpy(), B, topk, idx=gi, cnt=gc)
+    _check_out(to_f64(out), ref, dtype)
+
+
+def test_decode_all_blocks_equals_dense_row(ssa):
+    q, Kc, Vc, L = planted_decode(2, 8, 2, 777, 128, 64, 0, seed=9, dtype="bf16",
+                                  seqlens=[777, 400])
+    Kd = Kc.to(DEV)
+    S = ssa.ssa_block_summary(Kd, 64)
+    out, _ = ssa.ssa_decode(q.to(DEV), Kd, Vc.to(DEV), S, L.to(DEV), 64, 1 << 30)
+    for b, Lb in enumerate([777, 400]):
+        k = torch.from_numpy(to_f64(Kc[b, :, :Lb])).repeat_interleave(4, 0)
+        v = torch.from_numpy(to_f64(Vc[b, :, :Lb])).repeat_interleave(4, 0)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(to_f64(q[b]))[:, None, :], k, v)[:, 0].numpy()
+        _check_out(to_f64(out[b]), ref, "bf16")
+
+
+def test_decode_invalid_seqlen_writes_zeros(ssa):
+    q, Kc, Vc, _ = planted_decode(2, 4, 2, 256, 64, 64, 0, seed=10, dtype="f32")
+    L = torch.tensor([0, 256], dtype=torch.int32, device=DEV)
+    Kd = Kc.to(DEV)
+    S = ssa.ssa_block_summary(Kd, 64)
+    out, idx = ssa.ssa_decode(q.to(DEV), Kd, Vc.to(DEV), S, L, 64, 2)
+    assert torch.all(out[0] == 0)
+    assert torch.all(idx[0] == -1)
+    assert torch.isfinite(out[1]).all()
+
+
+def test_no_device_error_after_runs(ssa):
+    assert ssa.ssa_device_error() == 0
