@@ -208,3 +208,32 @@ def prefill(Q, K, V, B: int, topk: int, scale: float | None = None, stream=None)
     idx, cnt = ssa_route(Q, S, B, topk, K.shape[1], stream=stream)
     O, lse = ssa_sparse_attn_fwd(Q, K, V, idx, cnt, B, scale=scale, stream=stream)
     return O, lse, idx, cnt, S
+
+
+def ssa_decode_noalloc(q, Kc, Vc, S, seqlens, B: int, topk: int, scale: float | None = None,
+                       O=None, idx=None, want_idx: bool = True, stream=None):
+    """ssa_decode with the library's fixed scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory at call time.  Returns
+    ``(O, idx)`` like ``ssa_decode``.
+    """
+    for t, n in ((q, "q"), (Kc, "Kc"), (Vc, "Vc"), (seqlens, "seqlens")):
+        _need(t, n)
+    lib = load_library()
+    fn = lib.ssa_decode_noalloc
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp]
+    fn.restype = i
+    batch, Hq, d = q.shape
+    Hkv, Lmax = Kc.shape[1], Kc.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(q)
+    if idx is None and want_idx:
+        idx = torch.empty(batch, Hkv, decode_width(Lmax, B, topk), dtype=torch.int32,
+                          device=q.device)
+    _check("ssa_decode_noalloc", fn(
+        _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(S), _ptr(seqlens), batch, Hq, Hkv, Lmax,
+        d, B, topk, ctypes.c_float(scale), _ptr(O), _ptr(idx), _stream(stream)))
+    return O, idx

@@ -163,6 +163,38 @@ ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype d
                       size_t ws_bytes, ssa_stream stream);
 
 /*
+ * Largest scratch area ssa_decode_noalloc can use (40 MiB).
+ */
+#define SSA_DECODE_NOALLOC_MAX_BYTES ((size_t)40 << 20)
+
+/*
+ * ssa_decode without a caller-supplied workspace.  The pages have no
+ * counterpart: this is a library convenience.
+ *
+ * For callers that cannot allocate device memory at call time: code whose
+ * device memory is owned by another allocator it cannot reach, fixed-budget
+ * plug-in hosts, and serving loops where cudaMalloc (which may synchronise the
+ * device) is not allowed.  Arguments and results are those of ssa_decode
+ * minus `workspace` / `ws_bytes`; the scratch lives in one fixed device array
+ * of SSA_DECODE_NOALLOC_MAX_BYTES inside the library, which every GPU that
+ * loads the library holds until the process exits.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - The first call on each device looks up that device's address of the array
+ *   (with the device current), so make that first call before any stream
+ *   capture; later calls only read the cached address.
+ * - All calls share the one array and it keeps the previous call's contents;
+ *   everything that must start at zero is cleared by the call itself.  Calls
+ *   that overlap on the GPU (other streams, other host threads) race on it:
+ *   order them.
+ * - SSA_ERR_UNSUPPORTED if ssa_decode_workspace_size for these sizes exceeds
+ *   SSA_DECODE_NOALLOC_MAX_BYTES (checked on the host; nothing is launched).
+ */
+ssa_status ssa_decode_noalloc(const void* q, const void* Kc, const void* Vc, ssa_dtype dtype,
+                              const float* S, const int32_t* seqlens, int batch, int Hq, int Hkv,
+                              int Lmax, int d, int B, int topk, float scale, void* O,
+                              int32_t* idx, ssa_stream stream);
+
+/*
  * Device error word: 0, or the ssa_status of the first bounded device-side
  * wait that expired since the last reset.  Synchronises the device, then
  * writes the word to *code and resets it to 0.
