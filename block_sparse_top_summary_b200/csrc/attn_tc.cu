@@ -1,15 +1,484 @@
-// Stage 2 on the tensor cores (placeholder until the tcgen05 kernel lands).
+// Stage 2 on the tensor cores: exact softmax attention over the selected KV
+// blocks (SSA page, "2. Metodologia", sparse stream; DashAttention page,
+// "Estágio 2", a FlashAttention-style kernel iterating only the active blocks,
+// here written for sm_100a).
+//
+// Work item (one CTA): 256 query rows that share one block selection, i.e.
+// (batch, KV head g, query block i, group of 256/B query heads of g).  They
+// form two M-tiles of 128 rows (B = 64: two heads x 64 rows; B = 128: one head
+// x 128 rows).  The selected blocks are visited in chunks of 128 keys (two
+// blocks at B = 64, one at B = 128; an odd last block is paired with an
+// all-zero out-of-range box whose keys are masked).
+//
+// Roles (320 threads, 10 warps):
+//   warp 0      TMA producer: Q once (8 boxes of 64 x 64 bf16, 128-byte swizzle),
+//               then K and V of every chunk into a 2-stage ring;
+//   warp 1      TMEM owner (512 columns) and MMA issuer (one thread):
+//               S_t = Q_t K^T  (tcgen05.mma kind::f16, M=128 N=128 K=16, A and B
+//               from shared memory), O_t += P_t V (A = P from TMEM, B = V from
+//               shared memory, MN-major);
+//   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: thread = row =
+//               TMEM lane; read S (tcgen05.ld), scale to the log2 domain, mask
+//               (only the last chunk holds the diagonal block), online softmax
+//               with lazy rescaling (O in TMEM is rescaled only when the row max
+//               grows by more than 2^8), write P as bf16 pairs back into the S
+//               columns (tcgen05.st), and finally normalise O and store it.
+// TMEM columns: S/P of tile t at 128 t, O of tile t at 256 + 128 t.
+// Every mbarrier wait is bounded in time; on expiry the CTA records
+// SSA_ERR_TIMEOUT in the device error word, stops issuing work, drains what it
+// issued and frees its TMEM.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace ssa {
 
-bool attn_tc_supported(ssa_dtype, int, int, int, int) { return false; }
+__device__ int g_attn_tc_error = 0;
 
-cudaError_t launch_attn_tc(const void*, const void*, const void*, const int32_t*, const int32_t*,
-                           int, int, int, int, int, int, float, void*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kNS = 2;                      // K/V pipeline stages
+constexpr uint32_t kQBytes = 65536;         // 2 tiles x 128 rows x 128 d x 2 B
+constexpr uint32_t kKVBytes = 32768;        // 128 keys x 128 d x 2 B (K or V)
+constexpr uint32_t kSmemBytes = kQBytes + 2 * kNS * kKVBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s per wait
+
+struct __align__(8) Shared {
+  uint64_t q_full;
+  uint64_t k_full[kNS];
+  uint64_t v_full[kNS];
+  uint64_t kv_empty[kNS];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int sel[1];  // selection of this work item (cnt entries)
+};
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
 
-int read_and_reset_attn_tc_error() { return 0; }
+// Bounded wait: false when the CTA aborted or the wait expired (then the CTA
+// aborts and the device error word is set).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitNs) {
+        *abort = 1;
+        atomicCAS(&g_attn_tc_error, 0, (int)SSA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the result is broadcast, so the
+// warp stays converged for the .sync.aligned tcgen05 instructions that follow.
+__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+
+// Shared-memory matrix descriptor: 128-byte swizzle, sm_100 version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, M = 128, N = 128.
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) |
+                              ((128u >> 4) << 24);
+constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);  // B (= V) MN-major
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+}  // namespace
+
+template <int B>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
+    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
+    int Hq, int Hkv, int N, int nq, int max_sel, float scale_log2) {
+  constexpr int HPT = 128 / B;      // query heads per M-tile
+  constexpr int HPI = 2 * HPT;      // query heads per work item
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* Qs = base;
+  unsigned char* Ks = base + kQBytes;
+  unsigned char* Vs = Ks + kNS * kKVBytes;
+  Shared* sh = reinterpret_cast<Shared*>(Vs + kNS * kKVBytes);
+
+  const int G = Hq / Hkv;
+  const int subs = G / HPI;
+  const int bg = blockIdx.y;
+  const int b = bg / Hkv;
+  const int g = bg - b * Hkv;
+  const int i = nq - 1 - (int)(blockIdx.x / subs);
+  const int sub = blockIdx.x % subs;
+  const int h0 = g * G + sub * HPI;  // first query head of this work item
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ns = cnt[(int64_t)bg * nq + i];
+  // cnt >= 1 for any routing output (block 0 is always selected); a zero
+  // count makes the CTA skip all work and leave its rows unwritten.
+  const int nch = ns <= 0 ? 0 : (B == 64) ? (ns + 1) / 2 : ns;
+  volatile int* abort = &sh->abort;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&sh->q_full, 1);
+    for (int s = 0; s < kNS; ++s) {
+      ptx::mbar_init(&sh->k_full[s], 1);
+      ptx::mbar_init(&sh->v_full[s], 1);
+      ptx::mbar_init(&sh->kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(&sh->s_full[t], 1);
+      ptx::mbar_init(&sh->p_full[t], 128);
+      ptx::mbar_init(&sh->o_done[t], 1);
+    }
+    ptx::mbar_init(&sh->drain, 1);
+    sh->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  for (int s = threadIdx.x; s < ns; s += kThreads)
+    sh->sel[s] = idx[((int64_t)bg * nq + i) * max_sel + s];
+  if (warp == 1) {
+    ptx::tmem_alloc(&sh->tmem_base, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nch > 0) {
+      ptx::prefetch_tmap(&tmQ);
+      ptx::prefetch_tmap(&tmK);
+      ptx::prefetch_tmap(&tmV);
+      ptx::mbar_arrive_expect_tx(&sh->q_full, kQBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int hh = 0; hh < HPT; ++hh)
+          for (int rg = 0; rg < B / 64; ++rg)
+            for (int c = 0; c < 2; ++c)
+              ptx::tma_load_3d(Qs + t * 32768 + c * 16384 + (hh * B + rg * 64) * 128, &tmQ,
+                               c * 64, i * B + rg * 64, b * Hq + h0 + t * HPT + hh, &sh->q_full);
+      int issued = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % kNS;
+        if (c >= kNS && !wait_bar(&sh->kv_empty[s], ((c / kNS) - 1) & 1, abort)) break;
+        int y[2];
+        for (int kg = 0; kg < 2; ++kg) {
+          if (B == 64) {
+            const int p = 2 * c + kg;
+            y[kg] = p < ns ? sh->sel[p] * 64 : nq * B;  // past the end: zero box
+          } else {
+            y[kg] = sh->sel[c] * 128 + kg * 64;
+          }
+        }
+        ptx::mbar_arrive_expect_tx(&sh->k_full[s], kKVBytes);
+        for (int kg = 0; kg < 2; ++kg)
+          for (int cc = 0; cc < 2; ++cc)
+            ptx::tma_load_3d(Ks + s * kKVBytes + cc * 16384 + kg * 8192, &tmK, cc * 64, y[kg],
+                             b * Hkv + g, &sh->k_full[s]);
+        ptx::mbar_arrive_expect_tx(&sh->v_full[s], kKVBytes);
+        for (int kg = 0; kg < 2; ++kg)
+          for (int cc = 0; cc < 2; ++cc)
+            ptx::tma_load_3d(Vs + s * kKVBytes + cc * 16384 + kg * 8192, &tmV, cc * 64, y[kg],
+                             b * Hkv + g, &sh->v_full[s]);
+        issued = c + 1;
+      }
+      if (*abort) {
+        // let every issued copy land before the CTA's shared memory goes away
+        for (int c = (issued > kNS ? issued - kNS : 0); c < issued; ++c) {
+          const int s = c % kNS;
+          const uint32_t ph = (c / kNS) & 1;
+          volatile int no_abort = 0;
+          wait_bar(&sh->k_full[s], ph, &no_abort);
+          wait_bar(&sh->v_full[s], ph, &no_abort);
+        }
+        volatile int no_abort = 0;
+        wait_bar(&sh->q_full, 0, &no_abort);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t qa = ptx::smem_u32(Qs);
+      const uint32_t ka = ptx::smem_u32(Ks);
+      const uint32_t va = ptx::smem_u32(Vs);
+      bool ok = nch > 0 && wait_bar(&sh->q_full, 0, abort) && wait_bar(&sh->k_full[0], 0, abort);
+      bool any = false;
+      auto issue_qk = [&](int t, int s) {
+        ptx::tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::mma_ss(tmem + t * 128, sdesc(qa + t * 32768 + off, 16, 1024),
+                      sdesc(ka + s * kKVBytes + off, 16, 1024), kIdescQK, kk > 0);
+        }
+        ptx::mma_commit(&sh->s_full[t]);
+      };
+      auto issue_pv = [&](int t, int s, int c) {
+        ptx::tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk)
+          ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                      sdesc(va + s * kKVBytes + kk * 2048, 16384, 1024), kIdescPV,
+                      (c > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(&sh->o_done[t]);
+      };
+      if (ok) {
+        issue_qk(0, 0);
+        issue_qk(1, 0);
+        any = true;
+      }
+      for (int c = 0; ok && c < nch; ++c) {
+        const int s = c % kNS;
+        const uint32_t ph = (c / kNS) & 1;
+        if (!(ok = wait_bar(&sh->v_full[s], ph, abort))) break;
+        if (!(ok = wait_bar(&sh->p_full[0], c & 1, abort))) break;
+        issue_pv(0, s, c);
+        const bool more = c + 1 < nch;
+        const int s1 = (c + 1) % kNS;
+        if (more) {
+          if (!(ok = wait_bar(&sh->k_full[s1], ((c + 1) / kNS) & 1, abort))) break;
+          issue_qk(0, s1);
+        }
+        if (!(ok = wait_bar(&sh->p_full[1], c & 1, abort))) break;
+        issue_pv(1, s, c);
+        ptx::mma_commit(&sh->kv_empty[s]);
+        if (more) issue_qk(1, s1);
+      }
+      if (any) {
+        // every MMA issued by this thread has completed once `drain` flips
+        ptx::mma_commit(&sh->drain);
+        volatile int no_abort = 0;
+        wait_bar(&sh->drain, 0, &no_abort);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 2) >> 2;          // M-tile
+    const int quarter = warp & 3;           // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;      // row in the tile = TMEM lane
+    const int hh = r / B;
+    const int pos = i * B + (r % B);
+    const int h = h0 + t * HPT + hh;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nch; ++c) {
+      if (!(ok = warp_wait_bar(&sh->s_full[t], c & 1, abort))) break;
+      ptx::tc_fence_after();
+      // v holds S, then the scaled / masked logits (as float bits), then the
+      // bf16 pairs of P packed into its first 64 words.
+      uint32_t v[128];
+      ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+      ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+      ptx::tmem_wait_ld();
+      const bool last = (c == nch - 1);
+      int jb[2];
+      if (B == 64) {
+        jb[0] = sh->sel[2 * c];
+        jb[1] = (2 * c + 1 < ns) ? sh->sel[2 * c + 1] : -1;
+      } else {
+        jb[0] = jb[1] = sh->sel[c];
+      }
+      float rmax = -INFINITY;
+#pragma unroll
+      for (int n = 0; n < 128; ++n) {
+        float x = __uint_as_float(v[n]) * scale_log2;
+        if (last) {
+          const int kg = n >> 6;
+          const int kpos = (B == 64) ? jb[kg] * 64 + (n & 63) : jb[0] * 128 + n;
+          if (jb[kg] < 0 || kpos > pos) x = -INFINITY;
+        }
+        v[n] = __float_as_uint(x);
+        rmax = fmaxf(rmax, x);
+      }
+      const float m_new = fmaxf(m_used, rmax);
+      bool need = false;
+      float alpha = 1.0f;
+      if (c == 0) {
+        m_used = m_new;
+      } else if (m_new > m_used + 8.0f) {
+        // lazy rescale: move the reference max only when it grew by > 2^8
+        need = true;
+        alpha = exp2f(m_used - m_new);
+        l *= alpha;
+        m_used = m_new;
+      }
+      float lsum = 0.f;
+#pragma unroll
+      for (int n = 0; n < 128; n += 2) {
+        const float p0 = exp2f(__uint_as_float(v[n]) - m_used);
+        const float p1 = exp2f(__uint_as_float(v[n + 1]) - m_used);
+        lsum += p0 + p1;
+        v[n >> 1] = pack_bf16(p0, p1);
+      }
+      l += lsum;
+      ptx::tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
+      ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
+      if (__any_sync(0xffffffffu, need)) {
+        // O must hold PV of the previous chunk before it is rescaled; PV of
+        // this chunk is not issued before this thread arrives on p_full.
+        if (!(ok = warp_wait_bar(&sh->o_done[t], (c - 1) & 1, abort))) break;
+        ptx::tc_fence_after();
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(tO + q * 32, ov);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          ptx::tmem_st32(tO + q * 32, ov);
+        }
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&sh->p_full[t]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && nch > 0 && warp_wait_bar(&sh->o_done[t], (nch - 1) & 1, abort)) {
+      ptx::tc_fence_after();
+      const float inv = 1.0f / l;
+      const bool store = pos < N;
+      __nv_bfloat16* orow = O + (((int64_t)b * Hq + h) * N + (store ? pos : 0)) * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t ov[32];
+        ptx::tmem_ld32(tO + q * 32, ov);
+        ptx::tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      if (store && lse != nullptr)
+        lse[((int64_t)b * Hq + h) * N + pos] = (m_used + log2f(l)) * 0.69314718055994530942f;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [heads, rows, 128] bf16 viewed as a 3-D tensor (d, rows, heads); 64 x 64 boxes.
+bool make_map(CUtensorMap* m, const void* ptr, int rows, int heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)rows * 128 * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int B>
+cudaError_t launch_tc_t(const void* Q, const void* K, const void* V, const int32_t* idx,
+                        const int32_t* cnt, int batch, int Hq, int Hkv, int N, int max_sel,
+                        float scale, void* O, float* lse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, N, batch * Hq) || !make_map(&mk, K, N, batch * Hkv) ||
+      !make_map(&mv, V, N, batch * Hkv))
+    return cudaErrorInvalidValue;
+  const int nq = (N + B - 1) / B;
+  const int G = Hq / Hkv;
+  const int subs = G / (2 * (128 / B));
+  const size_t smem = 1024 + kSmemBytes + sizeof(Shared) + sizeof(int) * (size_t)max_sel;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<B>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(nq * subs, batch * Hkv);
+  attn_tc_kernel<B><<<grid, kThreads, smem, st>>>(mq, mk, mv, idx, cnt, (__nv_bfloat16*)O, lse,
+                                                  Hq, Hkv, N, nq, max_sel,
+                                                  scale * 1.4426950408889634f);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_tc_supported(ssa_dtype dt, int Hq, int Hkv, int d, int B) {
+  if (dt != SSA_BF16 || d != 128 || (B != 64 && B != 128)) return false;
+  if (Hkv <= 0 || Hq % Hkv != 0) return false;
+  return ((Hq / Hkv) * B) % 256 == 0;
+}
+
+cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const int32_t* idx,
+                           const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
+                           int max_sel, float scale, void* O, float* lse, cudaStream_t st) {
+  if (max_sel > 8192) return cudaErrorInvalidValue;
+  return B == 64 ? launch_tc_t<64>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, max_sel, scale, O, lse,
+                                   st)
+                 : launch_tc_t<128>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, max_sel, scale, O, lse,
+                                    st);
+}
+
+int read_and_reset_attn_tc_error() {
+  int v = 0;
+  cudaMemcpyFromSymbol(&v, g_attn_tc_error, sizeof(int));
+  const int z = 0;
+  cudaMemcpyToSymbol(g_attn_tc_error, &z, sizeof(int));
+  return v;
+}
 
 }  // namespace ssa
