@@ -25,7 +25,6 @@ import argparse
 import json
 import math
 import os
-import subprocess
 import sys
 import time
 
@@ -75,53 +74,56 @@ def load_peaks():
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and throttle reasons with NVML on a thread (every 5 ms)
+    while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, dev_index: int):
         self.dev = dev_index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{dev_index}.csv")
+        self.samples = []
+        self.thread = None
 
     def start(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = int(vis.split(",")[self.dev]) if vis and vis.split(",")[0].isdigit() else self.dev
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            self.nv = None
+            return
+        self.stop_flag = False
+
+        def run():
+            while not self.stop_flag:
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+                time.sleep(0.005)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        self.stop_flag = True
+        self.thread.join()
+        if not self.samples:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(mhz), "source": "nvml, 5 ms"}
 
 
 # ------------------------------------------------------------ distributed
@@ -392,6 +394,42 @@ def run_reference(args, world, rank):
     print(json.dumps(line))
 
 
+def run_ncu_case(case: str, launches: int):
+    """Run one kernel of the hot path `launches` times on a bounded workload
+    (a few GB on the device, working set above the 126 MB L2) for profiling:
+    summary / route / attn on the 32K prefill workload, decode on 16 of the 64
+    sequences of the decode workload."""
+    import block_sparse_top_summary_b200 as ssa
+    ssa.load_library()
+    dev = torch.device("cuda", 0)
+    if case == "decode":
+        cd = CONFIGS["decode"]
+        q, Kc, Vc, L = planted_decode(16, cd.Hq, cd.Hkv, cd.L, cd.d, cd.B, cd.clusters,
+                                      seed=cd.seed, dtype=cd.dtype, device=dev)
+        Sc = ssa.ssa_block_summary(Kc, cd.B)
+        torch.cuda.synchronize()
+        for _ in range(launches):
+            ssa.ssa_decode(q, Kc, Vc, Sc, L, cd.B, cd.topk)
+    else:
+        cp = CONFIGS["prefill32k"]
+        Q, K, V = planted_prefill(cp.batch, cp.Hq, cp.Hkv, cp.N, cp.d, cp.B, cp.clusters,
+                                  seed=cp.seed, dtype=cp.dtype)
+        Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+        S = ssa.ssa_block_summary(Kd, cp.B)
+        idx, cnt = ssa.ssa_route(Qd, S, cp.B, cp.topk, cp.Hkv)
+        torch.cuda.synchronize()
+        for _ in range(launches):
+            if case == "summary":
+                ssa.ssa_block_summary(Kd, cp.B, S=S)
+            elif case == "route":
+                ssa.ssa_route(Qd, S, cp.B, cp.topk, cp.Hkv, idx=idx, cnt=cnt)
+            else:
+                ssa.ssa_sparse_attn_fwd(Qd, Kd, Vd, idx, cnt, cp.B)
+    torch.cuda.synchronize()
+    assert ssa.ssa_device_error() == 0
+    print(f"ncu case {case}: {launches} launches done")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -400,7 +438,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", choices=["summary", "route", "attn", "decode"], default=None,
+                    help="run one kernel on a bounded workload for profiling, then exit")
+    ap.add_argument("--ncu-launches", type=int, default=2)
     args = ap.parse_args()
+    if args.ncu_case:
+        run_ncu_case(args.ncu_case, args.ncu_launches)
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":

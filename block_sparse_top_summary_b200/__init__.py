@@ -7,6 +7,7 @@ There is no CPU fallback: every call needs the built library and a CUDA device.
 from .abi import (  # noqa: F401
     SSAError,
     decode_width,
+    ssa_debug_wait_timeout,
     load_library,
     prefill,
     route_width,

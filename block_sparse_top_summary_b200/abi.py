@@ -237,3 +237,13 @@ def ssa_decode_noalloc(q, Kc, Vc, S, seqlens, B: int, topk: int, scale: float | 
         _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(S), _ptr(seqlens), batch, Hq, Hkv, Lmax,
         d, B, topk, ctypes.c_float(scale), _ptr(O), _ptr(idx), _stream(stream)))
     return O, idx
+
+
+# ------------------------------------------------------------- test hooks
+def ssa_debug_wait_timeout(limit_us: int, stream=None):
+    """Run the bounded-wait self-test (include/ssa_debug.h); read the result with
+    ssa_device_error()."""
+    fn = load_library().ssa_debug_wait_timeout
+    fn.argtypes = [ctypes.c_int, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check("ssa_debug_wait_timeout", fn(limit_us, _stream(stream)))

@@ -10,20 +10,23 @@
 // blocks at B = 64, one at B = 128; an odd last block is paired with an
 // all-zero out-of-range box whose keys are masked).
 //
-// Roles (320 threads, 10 warps):
+// Roles (576 threads, 18 warps):
 //   warp 0      TMA producer: Q once (8 boxes of 64 x 64 bf16, 128-byte swizzle),
 //               then K and V of every chunk into a 2-stage ring;
 //   warp 1      TMEM owner (512 columns) and MMA issuer (one thread):
 //               S_t = Q_t K^T  (tcgen05.mma kind::f16, M=128 N=128 K=16, A and B
 //               from shared memory), O_t += P_t V (A = P from TMEM, B = V from
 //               shared memory, MN-major);
-//   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: thread = row =
-//               TMEM lane; read S (tcgen05.ld), scale to the log2 domain, mask
-//               (only the last chunk holds the diagonal block), online softmax
-//               with lazy rescaling (O in TMEM is rescaled only when the row max
-//               grows by more than 2^8), write P as bf16 pairs back into the S
-//               columns (tcgen05.st), and finally normalise O and store it.
-// TMEM columns: S/P of tile t at 128 t, O of tile t at 256 + 128 t.
+//   warps 2-9   softmax of tile 0, warps 10-17 softmax of tile 1: two threads
+//               per row (row = TMEM lane, each thread one 64-key half); read S
+//               (tcgen05.ld), mask (only the last chunk holds the diagonal
+//               block), exchange the half-row maxima through shared memory,
+//               online softmax in the log2 domain with lazy rescaling (O in
+//               TMEM is rescaled only when the row max grows by more than 2^8),
+//               write P as bf16 pairs into the first 32 columns of the thread's
+//               own S half (tcgen05.st), and finally normalise O and store it.
+// TMEM columns: S of tile t at 128 t (P of keys 0-63 at 128 t, of keys 64-127
+// at 128 t + 64), O of tile t at 256 + 128 t.
 // Every mbarrier wait is bounded in time; on expiry the CTA records
 // SSA_ERR_TIMEOUT in the device error word, stops issuing work, drains what it
 // issued and frees its TMEM.
@@ -34,6 +37,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "ssa_debug.h"
 
 namespace ssa {
 
@@ -41,13 +45,14 @@ __device__ int g_attn_tc_error = 0;
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
 constexpr int kNS = 2;                      // K/V pipeline stages
 constexpr uint32_t kQBytes = 65536;         // 2 tiles x 128 rows x 128 d x 2 B
 constexpr uint32_t kKVBytes = 32768;        // 128 keys x 128 d x 2 B (K or V)
 constexpr uint32_t kSmemBytes = kQBytes + 2 * kNS * kKVBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s per wait
+
 
 struct __align__(8) Shared {
   uint64_t q_full;
@@ -58,6 +63,10 @@ struct __align__(8) Shared {
   uint64_t p_full[2];
   uint64_t o_done[2];
   uint64_t drain;
+  uint64_t mx_full[2];  // per tile: both half-row maxima of the chunk are written
+  uint64_t l_full[2];   // per tile: both half-row sums are written (epilogue)
+  float mx[2][2][2][128];  // [chunk parity][tile][half][row]
+  float lx[2][2][128];     // [tile][half][row]
   uint32_t tmem_base;
   int abort;
   int sel[1];  // selection of this work item (cnt entries)
@@ -71,14 +80,15 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 
 // Bounded wait: false when the CTA aborted or the wait expired (then the CTA
 // aborts and the device error word is set).
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                         unsigned long long limit_ns = kWaitNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort = 1;
         atomicCAS(&g_attn_tc_error, 0, (int)SSA_ERR_TIMEOUT);
         return false;
@@ -93,6 +103,7 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, vo
   int ok = 0;
   if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) ptx::mbar_try_wait(bar, parity);  // completed phase: gives every lane acquire order
   return ok != 0;
 }
 
@@ -107,10 +118,91 @@ constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) 
                               ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);  // B (= V) MN-major
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
+
+// 2^x on the special-function unit (flushes results below 2^-126 to 0; 2^-inf = 0).
+__device__ __forceinline__ float ex2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (a, b) = (a * s + c, b * s + c) with one packed f32x2 FMA; s2 = {s, s}, c2 = {c, c}.
+__device__ __forceinline__ void fma2(float& a, float& b, uint64_t s2, uint64_t c2) {
+  asm("{\n\t.reg .b64 x;\n\tmov.b64 x, {%0, %1};\n\tfma.rn.f32x2 x, x, %2, %3;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "l"(s2), "l"(c2));
+}
+
+// acc += {a, b} with one packed f32x2 add.
+__device__ __forceinline__ void add2(uint64_t& acc, float a, float b) {
+  asm("{\n\t.reg .b64 x;\n\tmov.b64 x, {%1, %2};\n\tadd.f32x2 %0, %0, x;\n\t}"
+      : "+l"(acc)
+      : "f"(a), "f"(b));
+}
+
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ float sum2(uint64_t r) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+  return a + b;
+}
+
+// bf16 pair {lo, hi} (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Max of 32 values (2 independent 3-input max chains) folded into m.
+__device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
+  float a0 = m, a1 = -INFINITY;
+#pragma unroll
+  for (int n = 0; n < 32; n += 4) {
+    a0 = max3f(a0, __uint_as_float(v[n]), __uint_as_float(v[n + 1]));
+    a1 = max3f(a1, __uint_as_float(v[n + 2]), __uint_as_float(v[n + 3]));
+  }
+  return fmaxf(a0, a1);
+}
+
+// Columns n (0..31) of a 32-column slice starting at column `col0` whose key is
+// masked (causal diagonal or the missing half of an odd chunk) become -inf.
+template <int B>
+__device__ __forceinline__ void mask32(uint32_t (&v)[32], int col0, const int (&lim)[2]) {
+#pragma unroll
+  for (int n = 0; n < 32; ++n) {
+    const int col = col0 + n;
+    const bool valid = (B == 64) ? ((col & 63) <= lim[col >> 6]) : (col <= lim[0]);
+    if (!valid) v[n] = __float_as_uint(-INFINITY);
+  }
+}
+
+// p = 2^(s * scale - m) for 32 raw scores, packed as 16 bf16 pairs into w;
+// adds the (fp32) p to acc.
+__device__ __forceinline__ void exp_pack32(const uint32_t (&v)[32], uint32_t (&w)[16], uint64_t s2,
+                                           uint64_t c2, uint64_t& acc) {
+#pragma unroll
+  for (int n = 0; n < 32; n += 2) {
+    float a = __uint_as_float(v[n]), b = __uint_as_float(v[n + 1]);
+    fma2(a, b, s2, c2);
+    a = ex2_mufu(a);
+    b = ex2_mufu(b);
+    add2(acc, a, b);
+    w[n >> 1] = cvt_bf16x2(a, b);
+  }
+}
+
 
 }  // namespace
 
@@ -155,10 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     }
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(&sh->s_full[t], 1);
-      ptx::mbar_init(&sh->p_full[t], 128);
+      ptx::mbar_init(&sh->p_full[t], 256);
       ptx::mbar_init(&sh->o_done[t], 1);
     }
     ptx::mbar_init(&sh->drain, 1);
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(&sh->mx_full[t], 256);
+      ptx::mbar_init(&sh->l_full[t], 256);
+    }
     sh->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -244,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       auto issue_pv = [&](int t, int s, int c) {
         ptx::tc_fence_after();
         for (int kk = 0; kk < 8; ++kk)
-          ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+          ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + (kk >> 2) * 64 + (kk & 3) * 8,
                       sdesc(va + s * kKVBytes + kk * 2048, 16384, 1024), kIdescPV,
                       (c > 0 || kk > 0) ? 1u : 0u);
         ptx::mma_commit(&sh->o_done[t]);
@@ -280,78 +376,118 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 2) >> 2;          // M-tile
+    const int t = (warp - 2) >> 3;          // M-tile
+    const int half = ((warp - 2) >> 2) & 1; // key half of the chunk: columns 64 half ..
     const int quarter = warp & 3;           // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;      // row in the tile = TMEM lane
     const int hh = r / B;
     const int pos = i * B + (r % B);
     const int h = h0 + t * HPT + hh;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128;
-    const uint32_t tO = tmem + lane_off + 256 + t * 128;
+    const uint32_t tS = tmem + lane_off + t * 128 + half * 64;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128 + half * 64;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int c = 0; c < nch; ++c) {
       if (!(ok = warp_wait_bar(&sh->s_full[t], c & 1, abort))) break;
       ptx::tc_fence_after();
-      // v holds S, then the scaled / masked logits (as float bits), then the
-      // bf16 pairs of P packed into its first 64 words.
-      uint32_t v[128];
-      ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
-      ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
-      ptx::tmem_wait_ld();
       const bool last = (c == nch - 1);
-      int jb[2];
-      if (B == 64) {
-        jb[0] = sh->sel[2 * c];
-        jb[1] = (2 * c + 1 < ns) ? sh->sel[2 * c + 1] : -1;
-      } else {
-        jb[0] = jb[1] = sh->sel[c];
-      }
-      float rmax = -INFINITY;
-#pragma unroll
-      for (int n = 0; n < 128; ++n) {
-        float x = __uint_as_float(v[n]) * scale_log2;
-        if (last) {
-          const int kg = n >> 6;
-          const int kpos = (B == 64) ? jb[kg] * 64 + (n & 63) : jb[0] * 128 + n;
-          if (jb[kg] < 0 || kpos > pos) x = -INFINITY;
+      // causal mask / missing block, only in the chunk holding the diagonal:
+      // key column n (0..127) of block half kg is valid iff (n mod 64) <=
+      // lim[kg] (B = 64), or n <= lim[0] (B = 128)
+      int lim[2] = {127, 127};
+      if (last) {
+        if (B == 64) {
+          for (int kg = 0; kg < 2; ++kg) {
+            const int p = 2 * c + kg;
+            const int j = p < ns ? sh->sel[p] : -1;
+            lim[kg] = j < 0 ? -1 : (j == i ? (r & 63) : 63);
+          }
+        } else {
+          lim[0] = lim[1] = (sh->sel[c] == i) ? r : 127;
         }
-        v[n] = __float_as_uint(x);
-        rmax = fmaxf(rmax, x);
       }
-      const float m_new = fmaxf(m_used, rmax);
+      // pass 1: this half's maximum, then the other half's through shared memory
+      float pm = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tS + q * 32, v);
+        ptx::tmem_wait_ld();
+        if (last) mask32<B>(v, half * 64 + q * 32, lim);
+        pm = max32(v, pm);
+      }
+      sh->mx[c & 1][t][half][r] = pm;
+      ptx::mbar_arrive(&sh->mx_full[t]);
+      // The two halves of a row must use one reference max.  From chunk 1 on,
+      // P is computed optimistically with the current reference m_used while
+      // the other half's maximum is in flight; the pass is redone only if the
+      // row max exceeds m_used by more than 2^kSlack (then P, l and O would
+      // leave a comfortable fp32 / bf16 range).  Chunk 0 waits for the
+      // exchange first.
+      constexpr float kSlack = 64.0f;
+      float rmax = -INFINITY;
+      bool have_rmax = false;
+      if (c == 0) {
+        if (!(ok = warp_wait_bar(&sh->mx_full[t], c & 1, abort))) break;
+        rmax = fmaxf(pm, sh->mx[c & 1][t][half ^ 1][r]) * scale_log2;
+        m_used = rmax;
+        have_rmax = true;
+      }
       bool need = false;
       float alpha = 1.0f;
-      if (c == 0) {
-        m_used = m_new;
-      } else if (m_new > m_used + 8.0f) {
-        // lazy rescale: move the reference max only when it grew by > 2^8
-        need = true;
-        alpha = exp2f(m_used - m_new);
-        l *= alpha;
-        m_used = m_new;
+      uint64_t acc = 0;
+      uint32_t w0[16], w1[16];  // P of this half, stored only once it is final
+      for (int attempt = 0; attempt < 2; ++attempt) {
+        const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+        const uint64_t s2 = pack2(scale_log2, scale_log2);
+        const uint64_t c2 = pack2(-mu, -mu);
+        // pass 2: p = 2^(s*scale - m) as bf16 pairs (S stays intact until the
+        // pairs are stored, so a redo can read it again)
+        acc = 0;
+        {
+          uint32_t v[32];
+          ptx::tmem_ld32(tS, v);
+          ptx::tmem_wait_ld();
+          if (last) mask32<B>(v, half * 64, lim);
+          exp_pack32(v, w0, s2, c2, acc);
+          ptx::tmem_ld32(tS + 32, v);
+          ptx::tmem_wait_ld();
+          if (last) mask32<B>(v, half * 64 + 32, lim);
+          exp_pack32(v, w1, s2, c2, acc);
+        }
+        if (!have_rmax) {
+          if (!(ok = warp_wait_bar(&sh->mx_full[t], c & 1, abort))) break;
+          rmax = fmaxf(pm, sh->mx[c & 1][t][half ^ 1][r]) * scale_log2;
+          have_rmax = true;
+        }
+        // both halves of a row see the same rmax and m_used, so they decide
+        // alike; the redo itself is warp-uniform (the loads and shuffles it
+        // runs are warp-collective), rows that do not need it recompute the
+        // same values
+        const bool my_need = attempt == 0 && c > 0 && rmax > m_used + kSlack;
+        if (my_need) {
+          need = true;
+          alpha = ex2_mufu(m_used - rmax);
+          l *= alpha;
+          m_used = rmax;
+        }
+        if (__any_sync(0xffffffffu, my_need)) continue;  // redo pass 2
+        break;
       }
-      float lsum = 0.f;
-#pragma unroll
-      for (int n = 0; n < 128; n += 2) {
-        const float p0 = exp2f(__uint_as_float(v[n]) - m_used);
-        const float p1 = exp2f(__uint_as_float(v[n + 1]) - m_used);
-        lsum += p0 + p1;
-        v[n >> 1] = pack_bf16(p0, p1);
-      }
-      l += lsum;
-      ptx::tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
-      ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
+      if (!ok) break;
+      // P words land on this half's first 32 S columns, all consumed by now
+      ptx::tmem_st16(tS, w0);
+      ptx::tmem_st16(tS + 16, w1);
+      if (!ok) break;
+      l += sum2(acc);
       if (__any_sync(0xffffffffu, need)) {
         // O must hold PV of the previous chunk before it is rescaled; PV of
         // this chunk is not issued before this thread arrives on p_full.
         if (!(ok = warp_wait_bar(&sh->o_done[t], (c - 1) & 1, abort))) break;
         ptx::tc_fence_after();
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           uint32_t ov[32];
           ptx::tmem_ld32(tO + q * 32, ov);
           ptx::tmem_wait_ld();
@@ -365,20 +501,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       ptx::mbar_arrive(&sh->p_full[t]);
     }
     // ------------------------------------------------------------ epilogue
+    if (ok && nch > 0) {
+      sh->lx[t][half][r] = l;
+      ptx::mbar_arrive(&sh->l_full[t]);
+      ok = warp_wait_bar(&sh->l_full[t], 0, abort);
+    }
     if (ok && nch > 0 && warp_wait_bar(&sh->o_done[t], (nch - 1) & 1, abort)) {
       ptx::tc_fence_after();
-      const float inv = 1.0f / l;
+      const float lrow = sh->lx[t][0][r] + sh->lx[t][1][r];
+      const float inv = 1.0f / lrow;
       const bool store = pos < N;
-      __nv_bfloat16* orow = O + (((int64_t)b * Hq + h) * N + (store ? pos : 0)) * 128;
+      __nv_bfloat16* orow = O + (((int64_t)b * Hq + h) * N + (store ? pos : 0)) * 128 + half * 64;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         uint32_t ov[32];
         ptx::tmem_ld32(tO + q * 32, ov);
         ptx::tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+          w[e] = cvt_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
@@ -386,8 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
             dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
       }
-      if (store && lse != nullptr)
-        lse[((int64_t)b * Hq + h) * N + pos] = (m_used + log2f(l)) * 0.69314718055994530942f;
+      if (store && half == 0 && lse != nullptr)
+        lse[((int64_t)b * Hq + h) * N + pos] = (m_used + log2f(lrow)) * 0.69314718055994530942f;
     }
   }
   ptx::tc_fence_before();
@@ -395,6 +537,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- test hooks
+// One thread waits on an mbarrier that nothing arrives on; the bounded wait
+// expires and records SSA_ERR_TIMEOUT.
+__global__ void wait_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+    abort_flag = 0;
+    wait_bar(&bar, 0, &abort_flag, limit_ns);
   }
 }
 
@@ -445,8 +601,8 @@ cudaError_t launch_tc_t(const void* Q, const void* K, const void* V, const int32
   const int G = Hq / Hkv;
   const int subs = G / (2 * (128 / B));
   const size_t smem = 1024 + kSmemBytes + sizeof(Shared) + sizeof(int) * (size_t)max_sel;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<B>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(nq * subs, batch * Hkv);
   attn_tc_kernel<B><<<grid, kThreads, smem, st>>>(mq, mk, mv, idx, cnt, (__nv_bfloat16*)O, lse,
@@ -482,3 +638,10 @@ int read_and_reset_attn_tc_error() {
 }
 
 }  // namespace ssa
+
+extern "C" ssa_status ssa_debug_wait_timeout(int limit_us, ssa_stream stream) {
+  if (limit_us < 1 || limit_us > 1000000) return SSA_ERR_INVALID_ARG;
+  ssa::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}

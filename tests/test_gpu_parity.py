@@ -241,3 +241,24 @@ def test_decode_invalid_seqlen_writes_zeros(ssa):
 
 def test_no_device_error_after_runs(ssa):
     assert ssa.ssa_device_error() == 0
+
+
+@pytest.mark.parametrize("B", [64, 128])
+def test_large_score_jump_in_a_later_block(ssa, B):
+    # Block 3 scores ~600 above the others (a log2-domain jump far beyond any
+    # lazy-rescale slack): the kernel must move its reference max and rescale
+    # the partial output, and still match the oracle.
+    torch.manual_seed(11)
+    N, d, Hq, Hkv = B * 8, 128, 8, 2
+    u = torch.nn.functional.normalize(torch.randn(d), dim=0)
+    Q = (u * 3.0).expand(1, Hq, N, d).clone() + 0.01 * torch.randn(1, Hq, N, d)
+    K = torch.randn(1, Hkv, N, d)
+    K[:, :, 3 * B:4 * B] = u * 200.0 + 0.1 * torch.randn(B, d)
+    V = torch.randn(1, Hkv, N, d)
+    Q, K, V = (x.to(torch.bfloat16).contiguous() for x in (Q, K, V))
+    out, lse, idx, cnt, _ = ssa.prefill(Q.to(DEV), K.to(DEV), V.to(DEV), B, 8)
+    gi = idx.cpu().numpy()
+    assert all(3 in gi[0, g, i, :cnt[0, g, i]] for g in range(Hkv) for i in range(4, 8))
+    ref, rlse = O.sparse_attention(to_f64(Q), to_f64(K), to_f64(V), gi, cnt.cpu().numpy(), B)
+    _check_out(to_f64(out), ref, "bf16")
+    assert np.max(np.abs(to_f64(lse) - rlse)) < 1e-2
