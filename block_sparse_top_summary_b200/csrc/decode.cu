@@ -46,11 +46,115 @@ __device__ __forceinline__ float reduce32_transpose(float (&v)[32]) {
   return v[0];
 }
 
+// Exclusive prefix sum of one int per thread over a 256-thread block.
+__device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int base = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const int x = wsum[w];
+    base += (w < warp) ? x : 0;
+    all += x;
+  }
+  __syncthreads();
+  *total = all;
+  return base + incl - v;
+}
+
+// Top-k by all 256 threads of the block over n scores in shared memory; same
+// result as warp_select_topk: the k highest scores, equal scores going to the
+// lower index, written ascending as first + e to out[0 ..).  4-pass MSB-first
+// radix select (8 bits per pass) on a shared histogram, then an index-ordered
+// compaction (block scans) of the keys above the threshold and the first
+// `need` keys equal to it.  Returns the number written.
+__device__ int block_select_topk(const float* sc, int n, int k, int first, int32_t* out,
+                                 uint32_t* hist, int* sbuf) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (k <= 0 || n <= 0) return 0;
+  if (k >= n) {
+    for (int e = t; e < n; e += 256) out[e] = first + e;
+    return n;
+  }
+  uint32_t prefix = 0, pmask = 0;
+  int need = k;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    hist[t] = 0;
+    __syncthreads();
+    for (int e = t; e < n; e += 256) {
+      const uint32_t key = order_key(sc[e]);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t c[8], local = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        c[q] = hist[255 - (lane * 8 + q)];
+        local += c[q];
+      }
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - local;
+      if (excl < (uint32_t)need && (uint32_t)need <= incl) {
+        uint32_t run = excl;
+        for (int q = 0; q < 8; ++q) {
+          if (run + c[q] >= (uint32_t)need) {
+            sbuf[8] = 255 - (lane * 8 + q);
+            sbuf[9] = (int)run;
+            break;
+          }
+          run += c[q];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= (uint32_t)sbuf[8] << shift;
+    pmask |= 255u << shift;
+    need -= sbuf[9];
+    __syncthreads();
+  }
+  // index-ordered compaction: thread t owns the contiguous range [e0, e1)
+  const int per = (n + 255) / 256;
+  const int e0 = min(t * per, n), e1 = min(e0 + per, n);
+  int neq = 0;
+  for (int e = e0; e < e1; ++e) neq += (order_key(sc[e]) == prefix);
+  int total;
+  int eqr = block_excl_scan(neq, sbuf, &total);
+  int ntake = 0;
+  for (int e = e0; e < e1; ++e) {
+    const uint32_t key = order_key(sc[e]);
+    if (key > prefix) ++ntake;
+    else if (key == prefix) ntake += (eqr++ < need);
+  }
+  int pos = block_excl_scan(ntake, sbuf, &total);
+  eqr = block_excl_scan(neq, sbuf, &total);  // recompute this thread's equal-key rank base
+  for (int e = e0; e < e1; ++e) {
+    const uint32_t key = order_key(sc[e]);
+    bool take = key > prefix;
+    if (key == prefix) take = (eqr++ < need);
+    if (take) out[pos++] = first + e;
+  }
+  return k;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- 1. route
 template <typename T, int D>
-__global__ void __launch_bounds__(256) decode_route_kernel(
+__global__ void __launch_bounds__(256, 2) decode_route_kernel(
     const T* __restrict__ q, const float* __restrict__ S, const int32_t* __restrict__ seqlens,
     int Hq, int Hkv, int Lmax, int B, int nsum, int kk, int width, int32_t* __restrict__ ws_idx,
     int32_t* __restrict__ ws_cnt, int* __restrict__ ws_ctr, int32_t* __restrict__ idx_out,
@@ -107,25 +211,23 @@ __global__ void __launch_bounds__(256) decode_route_kernel(
     }
   }
   __syncthreads();
-  if (warp == 0) {
-    int32_t* row = ws_idx + (int64_t)bg * width;
-    int n_sel = 0;
-    if (valid) {
-      n_sel = 1;
-      if (last >= 1) {
-        const int m = warp_select_topk(sc, n, kk, 1, row + 1, hist);
-        __syncwarp();
-        if (lane == 0) row[m + 1] = last;
-        n_sel = m + 2;
-      }
-      if (lane == 0) row[0] = 0;
+  __shared__ int sbuf[16];
+  int32_t* row = ws_idx + (int64_t)bg * width;
+  int n_sel = 0;
+  if (valid) {
+    n_sel = 1;
+    if (last >= 1) {
+      const int m = block_select_topk(sc, n, kk, 1, row + 1, hist, sbuf);
+      if (t == 0) row[m + 1] = last;
+      n_sel = m + 2;
     }
-    for (int p = n_sel + lane; p < width; p += 32) row[p] = -1;
-    if (lane == 0) ws_cnt[bg] = n_sel;
-    __syncwarp();
-    if (idx_out != nullptr) {
-      for (int p = lane; p < width; p += 32) idx_out[(int64_t)bg * width + p] = row[p];
-    }
+    if (t == 0) row[0] = 0;
+  }
+  for (int p = n_sel + t; p < width; p += 256) row[p] = -1;
+  if (t == 0) ws_cnt[bg] = n_sel;
+  __syncthreads();
+  if (idx_out != nullptr) {
+    for (int p = t; p < width; p += 256) idx_out[(int64_t)bg * width + p] = row[p];
   }
 }
 
@@ -137,7 +239,7 @@ __host__ __device__ constexpr int part_floats(int G) {
   return G * (D + 2);
 }
 
-template <typename T, int D>
+template <typename T, int D, int GP>
 __global__ void __launch_bounds__(256) decode_split_kernel(
     const T* __restrict__ q, const T* __restrict__ Kc, const T* __restrict__ Vc,
     const int32_t* __restrict__ seqlens, int Hq, int Hkv, int Lmax, int B, int width, int splits,
@@ -210,46 +312,60 @@ __global__ void __launch_bounds__(256) decode_split_kernel(
   __syncthreads();
 
   float* part = ws_part + ((int64_t)bg * splits + split) * part_floats<D>(G);
-  // ---- logits: thread per key, rotated 16-byte chunks to spread smem banks
-  constexpr int EPC = Vec16<T>::n;
-  constexpr int CPR = D / EPC;
-  float mloc[kMaxG];
+  // ---- logits, warp-cooperative: lane l holds d/32 coordinates of every head's
+  // q; a warp step takes 32/GP keys, so its 32 partial dot products (key x
+  // head) are reduced by one 31-shuffle butterfly that leaves dot product l
+  // in lane l.  Lane l always holds head l % GP.
+  constexpr int SL = D / 32;
+  constexpr int KPI = 32 / GP;
+  float qreg[GP][SL];
 #pragma unroll
-  for (int h = 0; h < kMaxG; ++h) mloc[h] = -INFINITY;
+  for (int h = 0; h < GP; ++h)
+#pragma unroll
+    for (int e = 0; e < SL; ++e) qreg[h][e] = (h < G) ? qs[h * D + lane * SL + e] : 0.f;
+  const int my_h = lane % GP;
+  float mymax = -INFINITY;
   if (ok) {
-    for (int k = t; k < nkeys; k += blockDim.x) {
-      float acc[kMaxG];
+    for (int k0 = warp * KPI; k0 < nkeys; k0 += 8 * KPI) {
+      float v[32];
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.f;
-      const T* kr = Ks + (size_t)k * D;
-      for (int c0 = 0; c0 < CPR; ++c0) {
-        const int c = (c0 + k) % CPR;
-        float f[EPC];
-        unpack16(*reinterpret_cast<const uint4*>(kr + c * EPC), f, (const T*)nullptr);
-#pragma unroll
-        for (int h = 0; h < kMaxG; ++h) {
-          if (h < G) {
-            const float* qh = qs + h * D + c * EPC;
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) acc[h] = fmaf(f[e], qh[e], acc[h]);
+      for (int kk = 0; kk < KPI; ++kk) {
+        const int k = min(k0 + kk, nkeys - 1);
+        float f[SL];
+        const T* kr = Ks + (size_t)k * D + lane * SL;
+        if constexpr (sizeof(T) == 2) {
+          if constexpr (SL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(kr);
+            bf16x2_to_f(w.x, f[0], f[1]);
+            bf16x2_to_f(w.y, f[2 % SL], f[3 % SL]);
+          } else {
+            bf16x2_to_f(*reinterpret_cast<const uint32_t*>(kr), f[0], f[1 % SL]);
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < SL; ++e) f[e] = reinterpret_cast<const float*>(kr)[e];
+        }
+#pragma unroll
+        for (int h = 0; h < GP; ++h) {
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < SL; ++e) a = fmaf(f[e], qreg[h][e], a);
+          v[kk * GP + h] = a;
         }
       }
-#pragma unroll
-      for (int h = 0; h < kMaxG; ++h) {
-        if (h < G) {
-          ps[k * kMaxG + h] = acc[h];
-          mloc[h] = fmaxf(mloc[h], acc[h]);
-        }
+      const float dot = reduce32_transpose(v);
+      const int k = k0 + lane / GP;
+      if (k < nkeys && my_h < G) {
+        ps[k * kMaxG + my_h] = dot;
+        mymax = fmaxf(mymax, dot);
       }
     }
   }
-  // CTA max per head
+  // CTA max per head: lanes of one head are lane % GP apart
 #pragma unroll
-  for (int h = 0; h < kMaxG; ++h) {
-    const float w = warp_max(mloc[h]);
-    if (lane == 0) red[warp * kMaxG + h] = w;
-  }
+  for (int o = 16; o >= GP; o >>= 1) mymax = fmaxf(mymax, __shfl_xor_sync(0xffffffffu, mymax, o));
+  if (lane < GP && lane < G) red[warp * kMaxG + lane] = mymax;
+  if (lane >= G && lane < kMaxG) red[warp * kMaxG + lane] = -INFINITY;
   __syncthreads();
   if (t < kMaxG) {
     float mm = -INFINITY;
@@ -365,9 +481,9 @@ DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int L
   p.nblk_max = (Lmax + B - 1) / B;
   p.kk = topk < p.nblk_max ? topk : p.nblk_max;
   p.width = p.kk + 2;
-  // about 32 KB of K+V per split (two 16 KB blocks at B=64, d=128, bf16)
+  // about 64 KB of K+V per split (two 32 KB blocks at B=64, d=128, bf16)
   const int blk_bytes = 2 * B * d * 2;
-  p.per_split = blk_bytes >= 32768 ? 1 : 32768 / blk_bytes;
+  p.per_split = blk_bytes >= 65536 ? 1 : 65536 / blk_bytes;
   p.splits = (p.width + p.per_split - 1) / p.per_split;
   const size_t bg = (size_t)batch * Hkv;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -406,13 +522,23 @@ static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const voi
   if (ored_floats > ps_floats) ps_floats = ored_floats;
   const size_t smem2 = 2 * (size_t)nk_max * D * sizeof(T) +
                        sizeof(float) * ((size_t)kMaxG * D + ps_floats + 9 * kMaxG);
-  e = cudaFuncSetAttribute(decode_split_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem2);
-  if (e != cudaSuccess) return e;
   dim3 grid(p.splits, batch * Hkv);
-  decode_split_kernel<T, D><<<grid, 256, smem2, st>>>(
-      (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, p.splits,
-      p.per_split, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O, scale * 1.4426950408889634f);
+  const float sl2 = scale * 1.4426950408889634f;
+  if (p.G <= 4) {
+    e = cudaFuncSetAttribute(decode_split_kernel<T, D, 4>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
+    if (e != cudaSuccess) return e;
+    decode_split_kernel<T, D, 4><<<grid, 256, smem2, st>>>(
+        (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, p.splits,
+        p.per_split, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O, sl2);
+  } else {
+    e = cudaFuncSetAttribute(decode_split_kernel<T, D, 8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
+    if (e != cudaSuccess) return e;
+    decode_split_kernel<T, D, 8><<<grid, 256, smem2, st>>>(
+        (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, p.splits,
+        p.per_split, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O, sl2);
+  }
   return cudaGetLastError();
 }
 

@@ -8,8 +8,9 @@
 //
 // One fused kernel, one CTA of 256 threads per (tile of 8 query blocks,
 // batch x KV head):
-//   1. pool: stream the tile's Q rows (G heads x B rows x d per query block)
-//      with coalesced 16-byte loads into 8 fp32 means qbar (HBM-bound part);
+//   1. pool: warp w streams query block w of the tile (G heads x B rows x d)
+//      with coalesced 16-byte loads, 16 in flight per lane, into its fp32
+//      mean qbar (the HBM-bound part);
 //   2. score: every warp takes 4 candidate summaries at a time; lane l holds
 //      d/32 coordinates of each summary and of the 8 qbar rows, so one
 //      coalesced load feeds 8*d/32 FMAs; the 32 partial dot products of a
@@ -58,12 +59,10 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
                                                     float inv_sqrt_d) {
   constexpr int EPC = Vec16<T>::n;
   constexpr int CPR = D / EPC;
-  constexpr int RL = 256 / CPR;
   constexpr int SL = D / 32;  // summary coordinates per lane
   extern __shared__ __align__(16) float smem[];
   float* qbar = smem;                                        // [TQ][D]
-  float* red = qbar + TQ * D;                                // [RL][D]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(red + RL * D);  // [TQ][256]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(qbar + TQ * D);  // [TQ][256]
   float* sc = reinterpret_cast<float*>(hist + TQ * 256);     // [TQ][sc_stride]
 
   const int t = threadIdx.x;
@@ -77,51 +76,57 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
   const int i0 = tile * TQ;
   const int i1 = min(i0 + TQ, nq);
 
-  // ---- 1. pool Q over (rows of the block) x (heads of the group)
+  // ---- 1. pool Q over (rows of the block) x (heads of the group): warp w
+  // pools query block i0 + w.  A warp load covers RPW whole rows (16-byte
+  // chunk cc of row rs); 16 loads are in flight per lane; rows meet by
+  // xor-shuffles at the end, so this phase needs no block barrier.
   {
-    const int cc = t % CPR;
-    const int rl = t / CPR;
-    for (int qi = i0; qi < i1; ++qi) {
+    constexpr int LPR = CPR < 32 ? CPR : 32;  // lanes per row
+    constexpr int RPW = 32 / LPR;             // rows per warp load
+    constexpr int U = 16;                     // loads in flight per lane
+    const int qi = i0 + warp;
+    if (qi < i1) {
       const int rows = min(B, N - qi * B);
       const int R = G * rows;
+      const int cc = lane % LPR;
+      const int rs = lane / LPR;
       float acc[EPC];
 #pragma unroll
       for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
       const T* blk = Q + ((int64_t)(b * Hq + g * G) * N + (int64_t)qi * B) * D + cc * EPC;
-      int rr = rl;
-      for (; rr + 3 * RL < R; rr += 4 * RL) {
-        uint4 v[4];
+      for (int r0 = rs; r0 < R; r0 += RPW * U) {
+        uint4 v[U];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r = rr + q * RL;
-          const int h = r / rows;
-          v[q] = ldg16_stream(blk + ((int64_t)h * N + (r - h * rows)) * D);
+        for (int u = 0; u < U; ++u) {
+          const int r = r0 + u * RPW;
+          if (r < R) {
+            const int h = r / rows;
+            v[u] = ldg16_stream(blk + ((int64_t)h * N + (r - h * rows)) * D);
+          } else {
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+          }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int u = 0; u < U; ++u) {
           float f[EPC];
-          unpack16(v[q], f, (const T*)nullptr);
+          unpack16(v[u], f, (const T*)nullptr);
 #pragma unroll
           for (int e = 0; e < EPC; ++e) acc[e] += f[e];
         }
       }
-      for (; rr < R; rr += RL) {
-        const int h = rr / rows;
-        float f[EPC];
-        unpack16(ldg16_stream(blk + ((int64_t)h * N + (rr - h * rows)) * D), f, (const T*)nullptr);
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) acc[e] += f[e];
-      }
+      for (int o = LPR; o < 32; o <<= 1)
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) red[rl * D + cc * EPC + e] = acc[e];
-      __syncthreads();
-      if (t < D) {
-        float s = 0.f;
-        for (int q = 0; q < RL; ++q) s += red[q * D + t];
-        qbar[(qi - i0) * D + t] = s / (float)R;
+        for (int e = 0; e < EPC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+      if (rs == 0) {
+        const float inv = 1.0f / (float)R;
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) qbar[warp * D + cc * EPC + e] = acc[e] * inv;
       }
-      __syncthreads();
     }
+    // CPR > 32 (fp32, d = 128 has CPR = 32): one row per warp load covers d
+    static_assert(CPR <= 32, "a row must fit one warp load");
+    __syncthreads();
   }
 
   // ---- 2. scores for candidates j = 1 .. i1-2 against all TQ rows
@@ -191,14 +196,11 @@ template <typename T, int D>
 static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int Hq, int Hkv, int N,
                                   int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
                                   cudaStream_t st) {
-  constexpr int EPC = Vec16<T>::n;
-  constexpr int RL = 256 / (D / EPC);
   const int nq = (N + B - 1) / B;
   const int nfull = N / B;
   const int ntiles = (nq + TQ - 1) / TQ;
   const int sc_stride = nq > 2 ? nq - 2 : 1;
-  const size_t smem = sizeof(float) * ((size_t)TQ * D + (size_t)RL * D + (size_t)TQ * 256 +
-                                       (size_t)TQ * sc_stride);
+  const size_t smem = sizeof(float) * ((size_t)TQ * D + (size_t)TQ * 256 + (size_t)TQ * sc_stride);
   cudaError_t e = cudaFuncSetAttribute(route_kernel<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
