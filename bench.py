@@ -127,15 +127,31 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ distributed
-def dist_setup(gpus: int):
+# The hot path partitions into independent problems: each rank runs the same
+# workloads on its own seeded inputs (weak scaling, no data-path collective).
+# torch.distributed is used only for the timing barrier and the max / sum of
+# per-rank numbers.
+def dist_setup(gpus: int, backend: str = "nccl"):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     return world, rank, local
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Seed of a rank's own problem."""
+    return base + rank
+
+
+def _reduce_device():
+    if torch.distributed.is_initialized() and torch.distributed.get_backend() == "nccl":
+        return "cuda"
+    return "cpu"
 
 
 def barrier(world):
@@ -146,7 +162,7 @@ def barrier(world):
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=_reduce_device(), dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -154,7 +170,7 @@ def max_over_ranks(x: float, world: int) -> float:
 def sum_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    t = torch.tensor([x], device=_reduce_device(), dtype=torch.float64)
     torch.distributed.all_reduce(t)
     return float(t.item())
 
@@ -171,11 +187,11 @@ def run_ours(args, world, rank, local):
 
     # --- inputs (seed offset by rank: each rank works on its own problem)
     Q, K, V = planted_prefill(cp.batch, cp.Hq, cp.Hkv, cp.N, cp.d, cp.B, cp.clusters,
-                              seed=cp.seed + rank, dtype=cp.dtype)
+                              seed=rank_seed(cp.seed, rank), dtype=cp.dtype)
     Qh, Kh, Vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
     q, Kc, Vc, L = planted_decode(cd.batch, cd.Hq, cd.Hkv, cd.L, cd.d, cd.B, cd.clusters,
-                                  seed=cd.seed + rank, dtype=cd.dtype, device=dev)
+                                  seed=rank_seed(cd.seed, rank), dtype=cd.dtype, device=dev)
     Sc = ssa.ssa_block_summary(Kc, cd.B)  # precomputed cache summaries (decode input)
     qh, Lh = q.cpu().pin_memory(), L.cpu().pin_memory()
 
