@@ -64,6 +64,25 @@ def decode_bytes(idx: np.ndarray, seqlens: np.ndarray, B: int, d: int, G: int, e
     return total
 
 
+def attn_traffic_per_launch():
+    """DRAM bytes (read + write) per attention launch from the committed ncu
+    record, or None when the kernel source changed since the capture."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", "attn_tc_prefill32k_traffic.txt")
+    src = os.path.join(ROOT, "block_sparse_top_summary_b200", "csrc", "attn_tc.cu")
+    if not (os.path.exists(rec) and os.path.exists(src)):
+        return None
+    kv = {}
+    for line in open(rec):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.strip().split("=", 1)
+            kv[k] = v
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if kv.get("kernel_source_sha256") != digest:
+        return None
+    return int(kv["dram_bytes_read"]) + int(kv["dram_bytes_write"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -309,7 +328,8 @@ def run_ours(args, world, rank, local):
     kernels["ssa_sparse_attn_fwd"]["frac_bf16"] = attn_tflops / bf16_peak
     roof = {"kernel": "ssa_sparse_attn_fwd", "bound": "tensor" if tc else "alu",
             "achieved": attn_tflops, "peak": bf16_peak, "unit": "TFLOP/s",
-            "frac": attn_tflops / bf16_peak, "traffic": None,
+            "frac": attn_tflops / bf16_peak, "traffic": attn_traffic_per_launch(),
+            "traffic_unit": "bytes per launch (ncu dram read+write, profiles/)",
             "peak_source": f"{peak_kind} bf16 dense (burst)",
             "work_per_launch": f"{flops:.4e} FLOP"}
 
@@ -449,7 +469,7 @@ def run_ncu_case(case: str, launches: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

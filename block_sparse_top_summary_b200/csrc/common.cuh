@@ -53,6 +53,24 @@ __device__ __forceinline__ uint4 ldg16_stream(const void* p) {
 __device__ __forceinline__ void store_out(float* p, float v) { *p = v; }
 __device__ __forceinline__ void store_out(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
+// acc += a * b on two fp32 lanes at once (one packed f32x2 FMA).
+__device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
+// Two bf16 (low half first) as a packed fp32 pair.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return ((uint64_t)(w & 0xffff0000u) << 32) | (uint64_t)(w << 16);
+}
+
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | (uint64_t)__float_as_uint(lo);
+}
+
+__device__ __forceinline__ float f32x2_sum(uint64_t v) {
+  return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
+}
+
 // Order-preserving map from fp32 to uint32: a > b (as floats, no NaN) iff key(a) > key(b).
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);

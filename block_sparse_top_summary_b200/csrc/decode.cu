@@ -246,6 +246,13 @@ __global__ void __launch_bounds__(256) decode_split_kernel(
     int per_split, const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
     float* __restrict__ ws_part, int* __restrict__ ws_ctr, T* __restrict__ O,
     float scale_log2) {
+  // logits layout: DL lanes per key, each holding DS coordinates of every
+  // head's q; a warp step covers KG keys
+  constexpr int DL = 8 * GP / 4;
+  constexpr int DS = D / DL;
+  constexpr int KG = 32 / DL;
+  // P.V layout: lane owns SL output coordinates of every head
+  constexpr int SL = D / 32;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int G = Hq / Hkv;
   const int split = blockIdx.x;
@@ -255,13 +262,12 @@ __global__ void __launch_bounds__(256) decode_split_kernel(
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int nk_max = per_split * B;  // keys this CTA can hold
 
-  // shared layout: K rows | V rows | qs[G][D] | p[nk_max][G] | red | bar
+  // shared layout: K rows | V rows | p[nk_max][GP] | ow[8][GP][D] | red
   T* Ks = reinterpret_cast<T*>(smem_raw);
   T* Vs = Ks + (size_t)nk_max * D;
-  float* qs = reinterpret_cast<float*>(Vs + (size_t)nk_max * D);
-  float* ps = qs + kMaxG * D;                  // [nk_max][kMaxG], later [4][kMaxG][D]
-  const size_t ps_floats = max((size_t)nk_max * kMaxG, (size_t)(256 / (D / 2)) * kMaxG * D);
-  float* red = ps + ps_floats;                 // [8][kMaxG] + [kMaxG]
+  float* ps = reinterpret_cast<float*>(Vs + (size_t)nk_max * D);
+  float* ow = ps + (size_t)nk_max * GP;
+  float* red = ow + (size_t)8 * GP * D;  // [8][GP] maxima / sums + [GP] totals
   __shared__ uint64_t bar;
   __shared__ int s_last;
 
@@ -301,149 +307,148 @@ __global__ void __launch_bounds__(256) decode_split_kernel(
       nkeys += min(B, L - j * B);
     }
   }
-  // queries, pre-scaled into the log2 domain
-  for (int e = t; e < G * D; e += blockDim.x) {
-    const int h = e / D;
-    qs[h * D + (e - h * D)] = (float)q[((int64_t)b * Hq + g * G + h) * D + (e - h * D)] * scale_log2;
-  }
+  // this lane's slice of every head's query, scaled into the log2 domain
+  const int kg = lane / DL, dl = lane % DL;
+  uint64_t qr[GP][DS / 2];
+#pragma unroll
+  for (int h = 0; h < GP; ++h)
+#pragma unroll
+    for (int e = 0; e < DS / 2; ++e) {
+      float lo = 0.f, hi = 0.f;
+      if (h < G) {
+        const T* qp = q + ((int64_t)b * Hq + g * G + h) * D + dl * DS + 2 * e;
+        lo = (float)qp[0] * scale_log2;
+        hi = (float)qp[1] * scale_log2;
+      }
+      qr[h][e] = f32x2(lo, hi);
+    }
   bool ok = true;
   if (s0 < s1) ok = ptx::mbar_wait_bounded(&bar, 0, kWaitLimit);
   if (!ok) atomicCAS(&g_decode_error, 0, (int)SSA_ERR_TIMEOUT);
   __syncthreads();
 
   float* part = ws_part + ((int64_t)bg * splits + split) * part_floats<D>(G);
-  // ---- logits, warp-cooperative: lane l holds d/32 coordinates of every head's
-  // q; a warp step takes 32/GP keys, so its 32 partial dot products (key x
-  // head) are reduced by one 31-shuffle butterfly that leaves dot product l
-  // in lane l.  Lane l always holds head l % GP.
-  constexpr int SL = D / 32;
-  constexpr int KPI = 32 / GP;
-  float qreg[GP][SL];
+  // ---- logits
+  float mx[GP];
+#pragma unroll
+  for (int h = 0; h < GP; ++h) mx[h] = -INFINITY;
+  if (ok) {
+    for (int k0 = warp * KG; k0 < nkeys; k0 += 8 * KG) {
+      const int k = k0 + kg;
+      const T* kr = Ks + (size_t)min(k, nkeys - 1) * D + dl * DS;
+      uint64_t acc[GP];
+#pragma unroll
+      for (int h = 0; h < GP; ++h) acc[h] = 0;
+#pragma unroll
+      for (int e = 0; e < DS / 2; ++e) {
+        uint64_t kv;
+        if constexpr (sizeof(T) == 2) {
+          kv = bf16x2_to_f32x2(reinterpret_cast<const uint32_t*>(kr)[e]);
+        } else {
+          kv = f32x2(reinterpret_cast<const float*>(kr)[2 * e],
+                     reinterpret_cast<const float*>(kr)[2 * e + 1]);
+        }
+#pragma unroll
+        for (int h = 0; h < GP; ++h) ffma2(acc[h], kv, qr[h][e]);
+      }
+      float a[GP];
+#pragma unroll
+      for (int h = 0; h < GP; ++h) a[h] = f32x2_sum(acc[h]);
+#pragma unroll
+      for (int o = 1; o < DL; o <<= 1)
+#pragma unroll
+        for (int h = 0; h < GP; ++h) a[h] += __shfl_xor_sync(0xffffffffu, a[h], o);
+      if (dl == 0 && k < nkeys) {
+#pragma unroll
+        for (int h = 0; h < GP; ++h) {
+          ps[k * GP + h] = a[h];
+          mx[h] = fmaxf(mx[h], a[h]);
+        }
+      }
+    }
+  }
+  // CTA max per head: lanes dl == 0 of the key groups, then the warps
+#pragma unroll
+  for (int o = DL; o < 32; o <<= 1)
+#pragma unroll
+    for (int h = 0; h < GP; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < GP; ++h) red[warp * GP + h] = mx[h];
+  }
+  __syncthreads();
+  if (t < GP) {
+    float mm = -INFINITY;
+    for (int w = 0; w < 8; ++w) mm = fmaxf(mm, red[w * GP + t]);
+    red[8 * GP + t] = mm;
+  }
+  __syncthreads();
+  // p = 2^(s - m) in place, per-thread sums
+  float lloc[GP];
+#pragma unroll
+  for (int h = 0; h < GP; ++h) lloc[h] = 0.f;
+  for (int k = t; k < nkeys; k += 256) {
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+      const float p = exp2f(ps[k * GP + h] - red[8 * GP + h]);
+      ps[k * GP + h] = p;
+      lloc[h] += p;
+    }
+  }
+  // ---- P.V: warp w walks keys w, w+8, ...; lane owns SL coordinates
+  uint64_t o2[GP][SL / 2];
 #pragma unroll
   for (int h = 0; h < GP; ++h)
 #pragma unroll
-    for (int e = 0; e < SL; ++e) qreg[h][e] = (h < G) ? qs[h * D + lane * SL + e] : 0.f;
-  const int my_h = lane % GP;
-  float mymax = -INFINITY;
-  if (ok) {
-    for (int k0 = warp * KPI; k0 < nkeys; k0 += 8 * KPI) {
-      float v[32];
+    for (int e = 0; e < SL / 2; ++e) o2[h][e] = 0;
+  __syncthreads();  // p complete
+  for (int k = warp; k < nkeys; k += 8) {
+    const T* vr = Vs + (size_t)k * D + lane * SL;
+    uint64_t vv[SL / 2];
 #pragma unroll
-      for (int kk = 0; kk < KPI; ++kk) {
-        const int k = min(k0 + kk, nkeys - 1);
-        float f[SL];
-        const T* kr = Ks + (size_t)k * D + lane * SL;
-        if constexpr (sizeof(T) == 2) {
-          if constexpr (SL == 4) {
-            const uint2 w = *reinterpret_cast<const uint2*>(kr);
-            bf16x2_to_f(w.x, f[0], f[1]);
-            bf16x2_to_f(w.y, f[2 % SL], f[3 % SL]);
-          } else {
-            bf16x2_to_f(*reinterpret_cast<const uint32_t*>(kr), f[0], f[1 % SL]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < SL; ++e) f[e] = reinterpret_cast<const float*>(kr)[e];
-        }
-#pragma unroll
-        for (int h = 0; h < GP; ++h) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < SL; ++e) a = fmaf(f[e], qreg[h][e], a);
-          v[kk * GP + h] = a;
-        }
-      }
-      const float dot = reduce32_transpose(v);
-      const int k = k0 + lane / GP;
-      if (k < nkeys && my_h < G) {
-        ps[k * kMaxG + my_h] = dot;
-        mymax = fmaxf(mymax, dot);
+    for (int e = 0; e < SL / 2; ++e) {
+      if constexpr (sizeof(T) == 2) {
+        vv[e] = bf16x2_to_f32x2(reinterpret_cast<const uint32_t*>(vr)[e]);
+      } else {
+        vv[e] = f32x2(reinterpret_cast<const float*>(vr)[2 * e],
+                      reinterpret_cast<const float*>(vr)[2 * e + 1]);
       }
     }
-  }
-  // CTA max per head: lanes of one head are lane % GP apart
 #pragma unroll
-  for (int o = 16; o >= GP; o >>= 1) mymax = fmaxf(mymax, __shfl_xor_sync(0xffffffffu, mymax, o));
-  if (lane < GP && lane < G) red[warp * kMaxG + lane] = mymax;
-  if (lane >= G && lane < kMaxG) red[warp * kMaxG + lane] = -INFINITY;
-  __syncthreads();
-  if (t < kMaxG) {
-    float mm = -INFINITY;
-    for (int w = 0; w < 8; ++w) mm = fmaxf(mm, red[w * kMaxG + t]);
-    red[8 * kMaxG + t] = mm;
-  }
-  __syncthreads();
-  // p = 2^(s - m), sums
-  float lloc[kMaxG];
+    for (int h = 0; h < GP; ++h) {
+      const float p = ps[k * GP + h];
+      const uint64_t p2 = f32x2(p, p);
 #pragma unroll
-  for (int h = 0; h < kMaxG; ++h) lloc[h] = 0.f;
-  for (int k = t; k < nkeys; k += blockDim.x) {
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-      if (h < G) {
-        const float p = exp2f(ps[k * kMaxG + h] - red[8 * kMaxG + h]);
-        ps[k * kMaxG + h] = p;
-        lloc[h] += p;
-      }
+      for (int e = 0; e < SL / 2; ++e) ffma2(o2[h][e], vv[e], p2);
     }
   }
-  __syncthreads();
 #pragma unroll
-  for (int h = 0; h < kMaxG; ++h) {
+  for (int h = 0; h < GP; ++h)
+#pragma unroll
+    for (int e = 0; e < SL / 2; ++e) {
+      ow[((size_t)warp * GP + h) * D + lane * SL + 2 * e] = __uint_as_float((uint32_t)o2[h][e]);
+      ow[((size_t)warp * GP + h) * D + lane * SL + 2 * e + 1] =
+          __uint_as_float((uint32_t)(o2[h][e] >> 32));
+    }
+  // row sums
+#pragma unroll
+  for (int h = 0; h < GP; ++h) {
     const float w = warp_sum(lloc[h]);
-    if (lane == 0) red[warp * kMaxG + h] = w;
+    if (lane == 0) red[warp * GP + h] = w;
   }
   __syncthreads();
   if (t < G) {
     float ll = 0.f;
-    for (int w = 0; w < 8; ++w) ll += red[w * kMaxG + t];
-    part[t] = red[8 * kMaxG + t];  // m
-    part[G + t] = ll;              // l
+    for (int w = 0; w < 8; ++w) ll += red[w * GP + t];
+    part[t] = red[8 * GP + t];  // m
+    part[G + t] = ll;           // l
   }
-  // o[h][d] = sum_k p[k][h] V[k][d]: thread owns a pair of coordinates and a
-  // quarter of the keys; quarters meet in shared memory (reusing ps's tail).
-  {
-    const int dp = t % (D / 2);
-    const int kq = t / (D / 2);
-    const int nq4 = 256 / (D / 2);
-    float acc[kMaxG][2];
+  for (int e = t; e < G * D; e += 256) {
+    const int h = e / D, dd = e - h * D;
+    float s = 0.f;
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) acc[h][0] = acc[h][1] = 0.f;
-    for (int k = kq; k < nkeys; k += nq4) {
-      float v0, v1;
-      if constexpr (sizeof(T) == 2) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(Vs + (size_t)k * D + 2 * dp);
-        bf16x2_to_f(w, v0, v1);
-      } else {
-        const float2 w = *reinterpret_cast<const float2*>(Vs + (size_t)k * D + 2 * dp);
-        v0 = w.x;
-        v1 = w.y;
-      }
-#pragma unroll
-      for (int h = 0; h < kMaxG; ++h) {
-        if (h < G) {
-          const float p = ps[k * kMaxG + h];
-          acc[h][0] = fmaf(p, v0, acc[h][0]);
-          acc[h][1] = fmaf(p, v1, acc[h][1]);
-        }
-      }
-    }
-    __syncthreads();  // everyone is done reading ps
-    float* ored = ps;  // [nq4][kMaxG][D]
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-      if (h < G) {
-        ored[((size_t)kq * kMaxG + h) * D + 2 * dp] = acc[h][0];
-        ored[((size_t)kq * kMaxG + h) * D + 2 * dp + 1] = acc[h][1];
-      }
-    }
-    __syncthreads();
-    for (int e = t; e < G * D; e += blockDim.x) {
-      const int h = e / D, dd = e - h * D;
-      float s = 0.f;
-      for (int z = 0; z < nq4; ++z) s += ored[((size_t)z * kMaxG + h) * D + dd];
-      part[2 * G + h * D + dd] = s;
-    }
+    for (int w = 0; w < 8; ++w) s += ow[((size_t)w * GP + h) * D + dd];
+    part[2 * G + h * D + dd] = s;
   }
   // ---- the last split of this (sequence, KV head) merges the partials
   __threadfence();
@@ -516,12 +521,9 @@ static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const voi
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nk_max = p.per_split * B;
-  const int nq4 = 256 / (D / 2);
-  size_t ps_floats = (size_t)nk_max * kMaxG;
-  const size_t ored_floats = (size_t)nq4 * kMaxG * D;
-  if (ored_floats > ps_floats) ps_floats = ored_floats;
+  const int GPv = p.G <= 4 ? 4 : 8;
   const size_t smem2 = 2 * (size_t)nk_max * D * sizeof(T) +
-                       sizeof(float) * ((size_t)kMaxG * D + ps_floats + 9 * kMaxG);
+                       sizeof(float) * ((size_t)nk_max * GPv + (size_t)8 * GPv * D + 9 * GPv);
   dim3 grid(p.splits, batch * Hkv);
   const float sl2 = scale * 1.4426950408889634f;
   if (p.G <= 4) {
