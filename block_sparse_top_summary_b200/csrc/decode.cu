@@ -10,14 +10,16 @@
 //      butterfly leaves dot product l in lane l), then one warp runs the exact
 //      radix top-k (ties to the lower index).  The block list goes to the
 //      scratch area (and to the caller's idx if given).
-//   2. split-KV attention: one CTA per (split, sequence, KV head).  Each split
-//      owns a contiguous run of the selected blocks; every block's K rows and
-//      V rows are contiguous in the BHND cache, so each is fetched with ONE
-//      untiled bulk copy (TMA) into shared memory, all issued up front on one
-//      mbarrier.  The CTA computes the G heads' logits, a local softmax
-//      (max m, sum l, unnormalised o) and writes that partial; the last CTA of
-//      a (sequence, KV head) to finish (atomic counter) merges the partials
-//      with a log-sum-exp combine and writes O.
+//   2. split-KV attention, a persistent streaming kernel (one CTA per SM).
+//      The selected blocks of all (sequence, KV head) pairs are cut into
+//      units of at most 32 KB of K + V rows; each CTA owns an equal
+//      contiguous run of units.  A producer warp fetches each unit's K rows
+//      and V rows (contiguous in the BHND cache) with one untiled bulk copy
+//      each into a ring of shared stages; sixteen consumer warps split every
+//      unit's keys and keep their own online softmax (max m, sum l,
+//      unnormalised o).  Where the run leaves a (sequence, KV head) the warps
+//      are merged; a pair split between CTAs is finished by the last of them
+//      (atomic counter) with a log-sum-exp combine of the partial records.
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -28,8 +30,6 @@ __device__ int g_decode_error = 0;
 
 namespace {
 
-constexpr int kMaxG = 8;            // query heads per KV head handled by the split kernel
-constexpr uint32_t kWaitLimit = 1u << 24;  // bounded mbarrier polls
 
 __device__ __forceinline__ float reduce32_transpose(float (&v)[32]) {
   const int lane = threadIdx.x & 31;
@@ -232,253 +232,536 @@ __global__ void __launch_bounds__(256, 2) decode_route_kernel(
 }
 
 // -------------------------------------------------------- 2. split-KV attention
-// Partial record per (sequence, KV head, split): m[G], l[G], o[G][D] (fp32,
+// Partial record per (sequence, KV head, part): m[G], l[G], o[G][D] (fp32,
 // log2 domain, o unnormalised).
 template <int D>
 __host__ __device__ constexpr int part_floats(int G) {
   return G * (D + 2);
 }
 
+namespace {
+
+constexpr int kCW = 16;                         // consumer warps
+constexpr int kMW = 8;                          // merge slots (consumer warps fold in pairs)
+constexpr int kStreamThreads = 32 * (kCW + 1);  // + one producer warp
+constexpr int kMaxStages = 8;
+constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s per bounded wait
+
+// Layout constants of the streaming kernel.
 template <typename T, int D, int GP>
-__global__ void __launch_bounds__(256) decode_split_kernel(
-    const T* __restrict__ q, const T* __restrict__ Kc, const T* __restrict__ Vc,
-    const int32_t* __restrict__ seqlens, int Hq, int Hkv, int Lmax, int B, int width, int splits,
-    int per_split, const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
-    float* __restrict__ ws_part, int* __restrict__ ws_ctr, T* __restrict__ O,
-    float scale_log2) {
-  // logits layout: DL lanes per key, each holding DS coordinates of every
-  // head's q; a warp step covers KG keys
-  constexpr int DL = 8 * GP / 4;
-  constexpr int DS = D / DL;
-  constexpr int KG = 32 / DL;
-  // P.V layout: lane owns SL output coordinates of every head
-  constexpr int SL = D / 32;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  const int G = Hq / Hkv;
-  const int split = blockIdx.x;
-  const int bg = blockIdx.y;
-  const int b = bg / Hkv;
-  const int g = bg - b * Hkv;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int nk_max = per_split * B;  // keys this CTA can hold
+struct StreamShape {
+  // logits: DL lanes per key, each holding DS coordinates of every head's
+  // query; a warp step covers KG keys.  A lane reads its coordinates as NV
+  // vectors of VB bytes at vector indices dl, dl + DL, ... of the row, so the
+  // DL lanes of a key read consecutive 16-byte words (no bank conflicts).
+  // After the reduction R lanes hold each head's dot product.
+  static constexpr int DL = 4 * GP < 32 ? 4 * GP : 32;
+  static constexpr int R = DL / GP;
+  static constexpr int KG = 32 / DL;
+  static constexpr int DS = D / DL;
+  static constexpr int VB = DS * (int)sizeof(T) < 16 ? DS * (int)sizeof(T) : 16;
+  static constexpr int EV = VB / (int)sizeof(T);
+  static constexpr int NV = DS / EV;
+  // P.V: lane owns SL consecutive output coordinates of every head
+  static constexpr int SL = D / 32;
+  // most keys of one unit (32 KB of K + V) and of one warp's share of it
+  static constexpr int CKM = 32768 / (2 * D * (int)sizeof(T));
+  static constexpr int KWM = CKM / kCW;
+  static_assert(KWM >= 1 && KWM <= 16, "per-warp scratch holds 16 keys");
+  // per-warp scratch: logits s[16][GP] | p pairs [16][GP] | alpha[GP] (+pad)
+  static constexpr int kPwBytes = 16 * GP * 4 + 16 * GP * 8 + 32;
+};
 
-  // shared layout: K rows | V rows | p[nk_max][GP] | ow[8][GP][D] | red
-  T* Ks = reinterpret_cast<T*>(smem_raw);
-  T* Vs = Ks + (size_t)nk_max * D;
-  float* ps = reinterpret_cast<float*>(Vs + (size_t)nk_max * D);
-  float* ow = ps + (size_t)nk_max * GP;
-  float* red = ow + (size_t)8 * GP * D;  // [8][GP] maxima / sums + [GP] totals
-  __shared__ uint64_t bar;
-  __shared__ int s_last;
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
-  const int L = seqlens[b];
-  const int ns = ws_cnt[bg];
-  const int s0 = split * per_split;
-  const int s1 = min(s0 + per_split, ns);
-  const int64_t kvbase = (int64_t)bg * Lmax;
-
-  // ---- issue every block's K and V bulk copies up front
-  int nkeys = 0;  // keys held, in selection order
-  if (s0 < s1) {
-    if (t == 0) {
-      ptx::mbar_init(&bar, 1);
-      ptx::fence_mbar_init();
-    }
-    __syncthreads();
-    if (t == 0) {
-      uint32_t total = 0;
-      for (int s = s0; s < s1; ++s) {
-        const int j = ws_idx[(int64_t)bg * width + s];
-        total += 2u * (uint32_t)(min(B, L - j * B) * D * (int)sizeof(T));
-      }
-      ptx::mbar_arrive_expect_tx(&bar, total);
-      int off = 0;
-      for (int s = s0; s < s1; ++s) {
-        const int j = ws_idx[(int64_t)bg * width + s];
-        const int rows = min(B, L - j * B);
-        const uint32_t bytes = (uint32_t)(rows * D * (int)sizeof(T));
-        ptx::bulk_g2s(Ks + (size_t)off * D, Kc + (kvbase + (int64_t)j * B) * D, bytes, &bar);
-        ptx::bulk_g2s(Vs + (size_t)off * D, Vc + (kvbase + (int64_t)j * B) * D, bytes, &bar);
-        off += rows;
+// Bounded wait by one thread: false when the CTA aborted or the wait expired
+// (then the CTA aborts and the device error word is set).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) {
+        *abort = 1;
+        atomicCAS(&g_decode_error, 0, (int)SSA_ERR_TIMEOUT);
+        return false;
       }
     }
-    for (int s = s0; s < s1; ++s) {
-      const int j = ws_idx[(int64_t)bg * width + s];
-      nkeys += min(B, L - j * B);
-    }
-  }
-  // this lane's slice of every head's query, scaled into the log2 domain
-  const int kg = lane / DL, dl = lane % DL;
-  uint64_t qr[GP][DS / 2];
-#pragma unroll
-  for (int h = 0; h < GP; ++h)
-#pragma unroll
-    for (int e = 0; e < DS / 2; ++e) {
-      float lo = 0.f, hi = 0.f;
-      if (h < G) {
-        const T* qp = q + ((int64_t)b * Hq + g * G + h) * D + dl * DS + 2 * e;
-        lo = (float)qp[0] * scale_log2;
-        hi = (float)qp[1] * scale_log2;
-      }
-      qr[h][e] = f32x2(lo, hi);
-    }
-  bool ok = true;
-  if (s0 < s1) ok = ptx::mbar_wait_bounded(&bar, 0, kWaitLimit);
-  if (!ok) atomicCAS(&g_decode_error, 0, (int)SSA_ERR_TIMEOUT);
-  __syncthreads();
-
-  float* part = ws_part + ((int64_t)bg * splits + split) * part_floats<D>(G);
-  // ---- logits
-  float mx[GP];
-#pragma unroll
-  for (int h = 0; h < GP; ++h) mx[h] = -INFINITY;
-  if (ok) {
-    for (int k0 = warp * KG; k0 < nkeys; k0 += 8 * KG) {
-      const int k = k0 + kg;
-      const T* kr = Ks + (size_t)min(k, nkeys - 1) * D + dl * DS;
-      uint64_t acc[GP];
-#pragma unroll
-      for (int h = 0; h < GP; ++h) acc[h] = 0;
-#pragma unroll
-      for (int e = 0; e < DS / 2; ++e) {
-        uint64_t kv;
-        if constexpr (sizeof(T) == 2) {
-          kv = bf16x2_to_f32x2(reinterpret_cast<const uint32_t*>(kr)[e]);
-        } else {
-          kv = f32x2(reinterpret_cast<const float*>(kr)[2 * e],
-                     reinterpret_cast<const float*>(kr)[2 * e + 1]);
-        }
-#pragma unroll
-        for (int h = 0; h < GP; ++h) ffma2(acc[h], kv, qr[h][e]);
-      }
-      float a[GP];
-#pragma unroll
-      for (int h = 0; h < GP; ++h) a[h] = f32x2_sum(acc[h]);
-#pragma unroll
-      for (int o = 1; o < DL; o <<= 1)
-#pragma unroll
-        for (int h = 0; h < GP; ++h) a[h] += __shfl_xor_sync(0xffffffffu, a[h], o);
-      if (dl == 0 && k < nkeys) {
-#pragma unroll
-        for (int h = 0; h < GP; ++h) {
-          ps[k * GP + h] = a[h];
-          mx[h] = fmaxf(mx[h], a[h]);
-        }
-      }
-    }
-  }
-  // CTA max per head: lanes dl == 0 of the key groups, then the warps
-#pragma unroll
-  for (int o = DL; o < 32; o <<= 1)
-#pragma unroll
-    for (int h = 0; h < GP; ++h) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o));
-  if (lane == 0) {
-#pragma unroll
-    for (int h = 0; h < GP; ++h) red[warp * GP + h] = mx[h];
-  }
-  __syncthreads();
-  if (t < GP) {
-    float mm = -INFINITY;
-    for (int w = 0; w < 8; ++w) mm = fmaxf(mm, red[w * GP + t]);
-    red[8 * GP + t] = mm;
-  }
-  __syncthreads();
-  // p = 2^(s - m) in place, per-thread sums
-  float lloc[GP];
-#pragma unroll
-  for (int h = 0; h < GP; ++h) lloc[h] = 0.f;
-  for (int k = t; k < nkeys; k += 256) {
-#pragma unroll
-    for (int h = 0; h < GP; ++h) {
-      const float p = exp2f(ps[k * GP + h] - red[8 * GP + h]);
-      ps[k * GP + h] = p;
-      lloc[h] += p;
-    }
-  }
-  // ---- P.V: warp w walks keys w, w+8, ...; lane owns SL coordinates
-  uint64_t o2[GP][SL / 2];
-#pragma unroll
-  for (int h = 0; h < GP; ++h)
-#pragma unroll
-    for (int e = 0; e < SL / 2; ++e) o2[h][e] = 0;
-  __syncthreads();  // p complete
-  for (int k = warp; k < nkeys; k += 8) {
-    const T* vr = Vs + (size_t)k * D + lane * SL;
-    uint64_t vv[SL / 2];
-#pragma unroll
-    for (int e = 0; e < SL / 2; ++e) {
-      if constexpr (sizeof(T) == 2) {
-        vv[e] = bf16x2_to_f32x2(reinterpret_cast<const uint32_t*>(vr)[e]);
-      } else {
-        vv[e] = f32x2(reinterpret_cast<const float*>(vr)[2 * e],
-                      reinterpret_cast<const float*>(vr)[2 * e + 1]);
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < GP; ++h) {
-      const float p = ps[k * GP + h];
-      const uint64_t p2 = f32x2(p, p);
-#pragma unroll
-      for (int e = 0; e < SL / 2; ++e) ffma2(o2[h][e], vv[e], p2);
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < GP; ++h)
-#pragma unroll
-    for (int e = 0; e < SL / 2; ++e) {
-      ow[((size_t)warp * GP + h) * D + lane * SL + 2 * e] = __uint_as_float((uint32_t)o2[h][e]);
-      ow[((size_t)warp * GP + h) * D + lane * SL + 2 * e + 1] =
-          __uint_as_float((uint32_t)(o2[h][e] >> 32));
-    }
-  // row sums
-#pragma unroll
-  for (int h = 0; h < GP; ++h) {
-    const float w = warp_sum(lloc[h]);
-    if (lane == 0) red[warp * GP + h] = w;
-  }
-  __syncthreads();
-  if (t < G) {
-    float ll = 0.f;
-    for (int w = 0; w < 8; ++w) ll += red[w * GP + t];
-    part[t] = red[8 * GP + t];  // m
-    part[G + t] = ll;           // l
-  }
-  for (int e = t; e < G * D; e += 256) {
-    const int h = e / D, dd = e - h * D;
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) s += ow[((size_t)w * GP + h) * D + dd];
-    part[2 * G + h * D + dd] = s;
-  }
-  // ---- the last split of this (sequence, KV head) merges the partials
-  __threadfence();
-  __syncthreads();
-  if (t == 0) s_last = (atomicAdd(&ws_ctr[bg], 1) == splits - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float* parts = ws_part + (int64_t)bg * splits * part_floats<D>(G);
-  for (int e = t; e < G * D; e += blockDim.x) {
-    const int h = e / D, dd = e - h * D;
-    T* op = O + ((int64_t)b * Hq + g * G + h) * D + dd;
-    if (ns == 0) {
-      store_out(op, 0.f);
-      continue;
-    }
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(parts + (int64_t)s * part_floats<D>(G) + h));
-    float num = 0.f, den = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float* ps_ = parts + (int64_t)s * part_floats<D>(G);
-      const float ms = __ldcg(ps_ + h);
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      den = fmaf(w, __ldcg(ps_ + G + h), den);
-      num = fmaf(w, __ldcg(ps_ + 2 * G + h * D + dd), num);
-    }
-    store_out(op, num / den);
   }
 }
+
+// Warp-uniform bounded wait: lane 0 polls, every lane then observes the
+// completed phase itself (acquire order for its own shared-memory reads).
+__device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_bounded(bar, parity, abort) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) ptx::mbar_try_wait(bar, parity);
+  return ok != 0;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+}
+
+template <int VB>
+__device__ __forceinline__ void ld_vec(const void* p, uint32_t (&w)[VB / 4]) {
+  if constexpr (VB == 16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (VB == 8) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x; w[1] = v.y;
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  }
+}
+
+// Words of T elements -> packed fp32 pairs.
+template <typename T, int NW>
+__device__ __forceinline__ void to_pairs(const uint32_t (&w)[NW], uint64_t* out) {
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int e = 0; e < NW; ++e) out[e] = bf16x2_to_f32x2(w[e]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < NW / 2; ++e) out[e] = ((uint64_t)w[2 * e + 1] << 32) | w[2 * e];
+  }
+}
+
+// CTA whose unit range [floor(x U / grid), floor((x+1) U / grid)) holds unit u.
+__device__ __forceinline__ int cta_of_unit(long long u, long long U, long long grid) {
+  return (int)(((u + 1) * grid + U - 1) / U - 1);
+}
+
+}  // namespace
+
+// Persistent streaming split-KV kernel.  The selected blocks of all
+// (sequence, KV head) pairs form one list of units (a unit is up to CK keys
+// of one block, K rows and V rows each contiguous in the cache); CTA x takes
+// the contiguous range [x U / grid, (x+1) U / grid) of that list, so every CTA
+// streams the same number of bytes.  Warp kCW issues one bulk copy for the K
+// rows and one for the V rows of each unit into a ring of `stages` shared
+// stages (full / empty mbarriers); the kCW consumer warps each take CK / kCW
+// keys of every unit and keep their own online softmax (m, l, o).  When the
+// range leaves a (sequence, KV head), the warps' states are merged; if the
+// pair lies wholly inside this CTA's range O is written directly, otherwise
+// the CTA writes a partial record and the last of the pair's CTAs (atomic
+// counter) merges the records with a log-sum-exp combine.
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
+    const T* __restrict__ q, const T* __restrict__ Kc, const T* __restrict__ Vc,
+    const int32_t* __restrict__ seqlens, int Hq, int Hkv, int Lmax, int B, int width, int CK,
+    int subs, int stages, int stage_bytes, long long U, int parts_max,
+    const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
+    float* __restrict__ ws_part, int* __restrict__ ws_ctr, T* __restrict__ O, float scale_log2) {
+  using SH = StreamShape<T, D, GP>;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
+  __shared__ int info[kMaxStages];  // rows held by each stage
+  __shared__ int s_abort, s_last;
+
+  const int G = Hq / Hkv;
+  const int Ubg = width * subs;
+  const long long grid = gridDim.x;
+  const long long u0 = (long long)blockIdx.x * U / grid;
+  const long long u1 = ((long long)blockIdx.x + 1) * U / grid;
+  const int nunits = (int)(u1 - u0);
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  volatile int* abort = &s_abort;
+
+  unsigned char* stage0 = smem_raw;
+  float* ow = reinterpret_cast<float*>(smem_raw + (size_t)stages * stage_bytes);  // [kMW][GP][D]
+  float* mw = ow + kMW * GP * D;                                                  // [kMW][GP]
+  float* lw = mw + kMW * GP;                                                      // [kMW][GP]
+  unsigned char* pwbase = reinterpret_cast<unsigned char*>(lw + kMW * GP);
+
+  if (t == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], kCW);
+    }
+    s_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kCW) {
+    // ------------------------------------------------------------ producer
+    // Lane i resolves unit base + i (block index, rows, cache offset); the
+    // next batch of 32 is resolved while this one is issued.
+    auto resolve = [&](long long u, long long& src, int& rows) {
+      src = 0;
+      rows = 0;
+      if (u >= u1) return;
+      const int bg = (int)(u / Ubg);
+      const int rem = (int)(u - (long long)bg * Ubg);
+      const int s = rem / subs, r = rem - s * subs;
+      if (s >= ws_cnt[bg]) return;
+      const int j = ws_idx[(int64_t)bg * width + s];
+      const int L = seqlens[bg / Hkv];
+      const int k0 = j * B + r * CK;
+      const int rr = min(CK, min(L, (j + 1) * B) - k0);
+      if (rr <= 0) return;
+      rows = rr;
+      src = ((int64_t)bg * Lmax + k0) * D;
+    };
+    long long src_n;
+    int rows_n;
+    resolve(u0 + lane, src_n, rows_n);
+    int issued = 0;
+    bool ok = true;
+    for (int base = 0; ok && base < nunits; base += 32) {
+      const long long src_c = src_n;
+      const int rows_c = rows_n;
+      resolve(u0 + base + 32 + lane, src_n, rows_n);
+      const int cnt = min(32, nunits - base);
+      for (int i = 0; i < cnt; ++i) {
+        const int n = base + i;
+        const int st = n % stages;
+        const long long src = __shfl_sync(0xffffffffu, src_c, i);
+        const int rows = __shfl_sync(0xffffffffu, rows_c, i);
+        if (n >= stages && !(ok = warp_wait_bounded(&empty[st], ((n / stages) - 1) & 1, abort)))
+          break;
+        if (lane == 0) {
+          info[st] = rows;
+          unsigned char* dst = stage0 + (size_t)st * stage_bytes;
+          if (rows > 0) {
+            const uint32_t bytes = (uint32_t)rows * D * (uint32_t)sizeof(T);
+            ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes);
+            ptx::bulk_g2s(dst, Kc + src, bytes, &full[st]);
+            ptx::bulk_g2s(dst + (size_t)CK * D * sizeof(T), Vc + src, bytes, &full[st]);
+          } else {
+            ptx::mbar_arrive(&full[st]);
+          }
+        }
+        issued = n + 1;
+      }
+    }
+    // every copy issued lands before the CTA may exit (also after an abort)
+    if (lane == 0) {
+      volatile int no_abort = 0;
+      for (int n = max(0, issued - stages); n < issued; ++n)
+        wait_bounded(&full[n % stages], (uint32_t)(n / stages) & 1u, &no_abort);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int kg = lane / SH::DL, dl = lane % SH::DL;
+  const int KW = CK / kCW;  // keys of each unit this warp takes (CK is a multiple of 16)
+  float* pws = reinterpret_cast<float*>(pwbase + warp * SH::kPwBytes);
+  uint64_t* pwp = reinterpret_cast<uint64_t*>(pwbase + warp * SH::kPwBytes + 16 * GP * 4);
+  float* pwa = reinterpret_cast<float*>(pwbase + warp * SH::kPwBytes + 16 * GP * 12);
+
+  uint64_t qr[GP][SH::DS / 2];
+  uint64_t o2[GP][SH::SL / 2];
+  float m_run = -INFINITY, l_run = 0.f;
+  int cur = -1;
+
+  for (int n = 0; n <= nunits; ++n) {
+    const int bg = n < nunits ? (int)((u0 + n) / Ubg) : -2;
+    if (bg != cur) {
+      if (cur >= 0) {
+        // ---- end of a (sequence, KV head): merge the warps' states.  Round
+        // 1: warps kMW.. publish, warp w < kMW folds in warp w + kMW; round 2:
+        // warps < kMW publish and every thread merges the kMW slots.
+        float l = l_run;
+#pragma unroll
+        for (int o = GP; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        const int slot = warp & (kMW - 1);
+        auto publish = [&]() {
+          if (lane < GP) {
+            mw[slot * GP + lane] = m_run;
+            lw[slot * GP + lane] = l;
+          }
+#pragma unroll
+          for (int h = 0; h < GP; ++h)
+#pragma unroll
+            for (int e = 0; e < SH::SL / 2; ++e)
+              *reinterpret_cast<uint64_t*>(ow + ((size_t)slot * GP + h) * D + lane * SH::SL + 2 * e) =
+                  o2[h][e];
+        };
+        if (warp >= kMW) publish();
+        consumer_sync();
+        if (warp < kMW) {
+          float m_new = m_run, l_new = l;
+#pragma unroll
+          for (int h = 0; h < GP; ++h) {
+            const float ma = __shfl_sync(0xffffffffu, m_run, h);  // lane h keeps head h
+            const float mb = mw[slot * GP + h];
+            const float M = fmaxf(ma, mb);
+            const float sa = ma == -INFINITY ? 0.f : ex2_approx(ma - M);
+            const float sb = mb == -INFINITY ? 0.f : ex2_approx(mb - M);
+#pragma unroll
+            for (int e = 0; e < SH::SL / 2; ++e) {
+              const uint64_t ob =
+                  *reinterpret_cast<const uint64_t*>(ow + ((size_t)slot * GP + h) * D + lane * SH::SL + 2 * e);
+              const float lo = __uint_as_float((uint32_t)o2[h][e]) * sa + __uint_as_float((uint32_t)ob) * sb;
+              const float hi = __uint_as_float((uint32_t)(o2[h][e] >> 32)) * sa +
+                               __uint_as_float((uint32_t)(ob >> 32)) * sb;
+              o2[h][e] = f32x2(lo, hi);
+            }
+            if (h == lane % GP) {
+              m_new = M;
+              l_new = l * sa + lw[slot * GP + h] * sb;
+            }
+          }
+          m_run = m_new;
+          l = l_new;
+          __syncwarp();
+          publish();
+        }
+        consumer_sync();
+        const int b = cur / Hkv, g = cur - b * Hkv;
+        const long long uf = (long long)cur * Ubg;
+        const int xf = cta_of_unit(uf, U, grid);
+        const int nparts = cta_of_unit(uf + Ubg - 1, U, grid) - xf + 1;
+        float* part = ws_part + ((int64_t)cur * parts_max + (blockIdx.x - xf)) * part_floats<D>(G);
+        for (int e = t; e < G * D; e += kCW * 32) {
+          const int h = e / D, dd = e - h * D;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kMW; ++w) M = fmaxf(M, mw[w * GP + h]);
+          float num = 0.f, den = 0.f;
+#pragma unroll
+          for (int w = 0; w < kMW; ++w) {
+            const float mwv = mw[w * GP + h];
+            if (mwv == -INFINITY) continue;
+            const float sc = exp2f(mwv - M);
+            num = fmaf(sc, ow[((size_t)w * GP + h) * D + dd], num);
+            den = fmaf(sc, lw[w * GP + h], den);
+          }
+          if (nparts == 1) {
+            store_out(O + ((int64_t)b * Hq + g * G + h) * D + dd, den > 0.f ? num / den : 0.f);
+          } else {
+            part[2 * G + h * D + dd] = num;
+            if (dd == 0) {
+              part[h] = M;
+              part[G + h] = den;
+            }
+          }
+        }
+        if (nparts > 1) __threadfence();
+        consumer_sync();
+        if (nparts > 1) {
+          if (t == 0) s_last = (atomicAdd(&ws_ctr[cur], 1) == nparts - 1);
+          consumer_sync();
+          if (s_last) {
+            __threadfence();
+            const float* parts = ws_part + (int64_t)cur * parts_max * part_floats<D>(G);
+            for (int e = t; e < G * D; e += kCW * 32) {
+              const int h = e / D, dd = e - h * D;
+              float M = -INFINITY;
+              for (int p = 0; p < nparts; ++p)
+                M = fmaxf(M, __ldcg(parts + (int64_t)p * part_floats<D>(G) + h));
+              float num = 0.f, den = 0.f;
+              for (int p = 0; p < nparts; ++p) {
+                const float* pp = parts + (int64_t)p * part_floats<D>(G);
+                const float mp = __ldcg(pp + h);
+                if (mp == -INFINITY) continue;
+                const float sc = exp2f(mp - M);
+                den = fmaf(sc, __ldcg(pp + G + h), den);
+                num = fmaf(sc, __ldcg(pp + 2 * G + h * D + dd), num);
+              }
+              store_out(O + ((int64_t)b * Hq + g * G + h) * D + dd, den > 0.f ? num / den : 0.f);
+            }
+          }
+        }
+      }
+      if (n == nunits) break;
+      // ---- start of a (sequence, KV head): its query slice, fresh state
+      cur = bg;
+      {
+        const int b = bg / Hkv, g = bg - b * Hkv;
+#pragma unroll
+        for (int h = 0; h < GP; ++h)
+#pragma unroll
+          for (int m = 0; m < SH::NV; ++m) {
+            uint64_t pr[SH::EV / 2];
+            if (h < G) {
+              uint32_t w[SH::VB / 4];
+              ld_vec<SH::VB>(q + ((int64_t)b * Hq + g * G + h) * D + (dl + SH::DL * m) * SH::EV, w);
+              to_pairs<T, SH::VB / 4>(w, pr);
+            } else {
+#pragma unroll
+              for (int e = 0; e < SH::EV / 2; ++e) pr[e] = 0;
+            }
+#pragma unroll
+            for (int e = 0; e < SH::EV / 2; ++e) {
+              const float lo = __uint_as_float((uint32_t)pr[e]) * scale_log2;
+              const float hi = __uint_as_float((uint32_t)(pr[e] >> 32)) * scale_log2;
+              qr[h][m * (SH::EV / 2) + e] = f32x2(lo, hi);
+            }
+          }
+#pragma unroll
+        for (int h = 0; h < GP; ++h)
+#pragma unroll
+          for (int e = 0; e < SH::SL / 2; ++e) o2[h][e] = 0;
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
+    }
+
+    // ---- one unit
+    const int st = n % stages;
+    if (warp_wait_bounded(&full[st], (uint32_t)(n / stages) & 1u, abort)) {
+      const int rows = info[st];
+      const int kw0 = warp * KW;
+      const int kwv = min(KW, rows - kw0);
+      if (kwv > 0) {
+        const T* Ks = reinterpret_cast<const T*>(stage0 + (size_t)st * stage_bytes);
+        const T* Vs = Ks + (size_t)CK * D;
+        // logits of this warp's keys, log2 domain.  The loops run to the
+        // compile-time maximum KWM with rows clamped into the unit, so they
+        // unroll and their shared loads overlap; keys >= kwv are masked.
+#pragma unroll
+        for (int sp = 0; sp < SH::KWM; sp += SH::KG) {
+          const int kl = sp + kg;
+          const bool valid = kl < kwv;
+          const T* kr = Ks + (size_t)(kw0 + min(kl, kwv - 1)) * D;
+          uint64_t acc[GP];
+#pragma unroll
+          for (int h = 0; h < GP; ++h) acc[h] = 0;
+#pragma unroll
+          for (int m = 0; m < SH::NV; ++m) {
+            uint32_t w[SH::VB / 4];
+            ld_vec<SH::VB>(kr + (dl + SH::DL * m) * SH::EV, w);
+            uint64_t kv[SH::EV / 2];
+            to_pairs<T, SH::VB / 4>(w, kv);
+#pragma unroll
+            for (int e = 0; e < SH::EV / 2; ++e)
+#pragma unroll
+              for (int h = 0; h < GP; ++h) ffma2(acc[h], kv[e], qr[h][m * (SH::EV / 2) + e]);
+          }
+          float a[GP];
+#pragma unroll
+          for (int h = 0; h < GP; ++h) a[h] = f32x2_sum(acc[h]);
+          // reduce-scatter over the DL lanes of the key: lane dl ends with
+          // head dl / R (the R lanes of a head hold the same sum)
+#pragma unroll
+          for (int c = GP, msk = SH::DL / 2; c > 1; c >>= 1, msk >>= 1) {
+            const bool upper = (dl & msk) != 0;
+#pragma unroll
+            for (int k = 0; k < c / 2; ++k) {
+              const float send = upper ? a[k] : a[k + c / 2];
+              const float keep = upper ? a[k + c / 2] : a[k];
+              a[k] = keep + __shfl_xor_sync(0xffffffffu, send, msk);
+            }
+          }
+          float s = a[0];
+#pragma unroll
+          for (int msk = SH::R / 2; msk >= 1; msk >>= 1) s += __shfl_xor_sync(0xffffffffu, s, msk);
+          if (dl % SH::R == 0) pws[kl * GP + dl / SH::R] = valid ? s : -INFINITY;
+        }
+        __syncwarp();
+        // online softmax: lane keeps head lane % GP; its elements are
+        // e = lane + 32 i (key e / GP)
+        constexpr int NEL = SH::KWM * GP;         // elements of the warp's keys
+        constexpr int NE = (NEL + 31) / 32;
+        float sv[NE];
+        float cm = -INFINITY;
+#pragma unroll
+        for (int i2 = 0; i2 < NE; ++i2) {
+          const int e = lane + 32 * i2;
+          sv[i2] = (NEL % 32 == 0 || e < NEL) ? pws[e] : -INFINITY;
+          cm = fmaxf(cm, sv[i2]);
+        }
+#pragma unroll
+        for (int o = GP; o < 32; o <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+        const float m_new = fmaxf(m_run, cm);          // finite: the warp has a valid key
+        const float alpha = ex2_approx(m_run - m_new);  // 0 on the first unit
+        l_run *= alpha;
+#pragma unroll
+        for (int i2 = 0; i2 < NE; ++i2) {
+          const float p = ex2_approx(sv[i2] - m_new);  // 0 for masked keys
+          l_run += p;
+          const int e = lane + 32 * i2;
+          if (NEL % 32 == 0 || e < NEL) pwp[e] = f32x2(p, p);
+        }
+        if (lane < GP) pwa[lane] = alpha;
+        m_run = m_new;
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < GP; ++h) {
+          const float al = pwa[h];
+#pragma unroll
+          for (int e = 0; e < SH::SL / 2; ++e) {
+            const float lo = __uint_as_float((uint32_t)o2[h][e]) * al;
+            const float hi = __uint_as_float((uint32_t)(o2[h][e] >> 32)) * al;
+            o2[h][e] = f32x2(lo, hi);
+          }
+        }
+        // P.V over this warp's keys (masked keys have p = 0 and are skipped)
+#pragma unroll
+        for (int kl = 0; kl < SH::KWM; ++kl) {
+          uint32_t w[SH::SL * (int)sizeof(T) / 4];
+          ld_vec<SH::SL * (int)sizeof(T)>(Vs + (size_t)(kw0 + min(kl, kwv - 1)) * D + lane * SH::SL,
+                                          w);
+          uint64_t vv[SH::SL / 2];
+          to_pairs<T, SH::SL * (int)sizeof(T) / 4>(w, vv);
+          const ulonglong2* pp = reinterpret_cast<const ulonglong2*>(pwp + kl * GP);
+          if (kl < kwv) {
+#pragma unroll
+            for (int h2 = 0; h2 < GP / 2; ++h2) {
+              const ulonglong2 p2 = pp[h2];
+#pragma unroll
+              for (int e = 0; e < SH::SL / 2; ++e) {
+                ffma2(o2[2 * h2][e], vv[e], p2.x);
+                ffma2(o2[2 * h2 + 1][e], vv[e], p2.y);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[st]);
+  }
+}
+
+namespace {
+
+// Unit geometry of the streaming kernel for one element size.
+struct StreamGeom {
+  int ck, subs, ubg;
+  long long units;
+  int parts_max;
+};
+
+constexpr int kStageTarget = 32768;  // bytes of K + V per stage
+constexpr int kGridMax = 512;        // upper bound on the streaming grid
+
+StreamGeom stream_geom(int bg, int width, int d, int B, int esize) {
+  StreamGeom s{};
+  int ck = kStageTarget / (2 * d * esize);
+  ck = ck < B ? ck : B;
+  s.ck = ck;
+  s.subs = (B + ck - 1) / ck;
+  s.ubg = width * s.subs;
+  s.units = (long long)bg * s.ubg;
+  // every CTA range holds at least lr units (grid <= kGridMax), so one
+  // (sequence, KV head) meets at most ceil(ubg / lr) + 1 ranges
+  const long long lr = s.units / kGridMax > 0 ? s.units / kGridMax : 1;
+  const long long pm = (s.ubg + lr - 1) / lr + 1;
+  s.parts_max = (int)(pm < s.ubg ? pm : s.ubg);
+  return s;
+}
+
+}  // namespace
 
 DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int Lmax) {
   DecodePlan p{};
@@ -486,18 +769,51 @@ DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int L
   p.nblk_max = (Lmax + B - 1) / B;
   p.kk = topk < p.nblk_max ? topk : p.nblk_max;
   p.width = p.kk + 2;
-  // about 64 KB of K+V per split (two 32 KB blocks at B=64, d=128, bf16)
-  const int blk_bytes = 2 * B * d * 2;
-  p.per_split = blk_bytes >= 65536 ? 1 : 65536 / blk_bytes;
-  p.splits = (p.width + p.per_split - 1) / p.per_split;
-  const size_t bg = (size_t)batch * Hkv;
+  const int bgn = batch * Hkv;
+  const StreamGeom s2 = stream_geom(bgn, p.width, d, B, 2);
+  const StreamGeom s4 = stream_geom(bgn, p.width, d, B, 4);
+  p.parts_max = s2.parts_max > s4.parts_max ? s2.parts_max : s4.parts_max;
+  const size_t bg = (size_t)bgn;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   p.off_idx = 0;
   p.off_cnt = up(p.off_idx + bg * p.width * sizeof(int32_t));
   p.off_ctr = up(p.off_cnt + bg * sizeof(int32_t));
   p.off_part = up(p.off_ctr + bg * sizeof(int32_t));
-  p.bytes = up(p.off_part + bg * p.splits * (size_t)p.G * (d + 2) * sizeof(float));
+  p.bytes = up(p.off_part + bg * p.parts_max * (size_t)p.G * (d + 2) * sizeof(float));
   return p;
+}
+
+template <typename T, int D, int GP>
+static cudaError_t launch_stream(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
+                                 const int32_t* seqlens, int batch, int Hq, int Hkv, int Lmax,
+                                 int B, float scale, void* O, int32_t* ws_idx, int32_t* ws_cnt,
+                                 int* ws_ctr, float* ws_part, cudaStream_t st) {
+  using SH = StreamShape<T, D, GP>;
+  const StreamGeom s = stream_geom(batch * Hkv, p.width, D, B, (int)sizeof(T));
+  const int stage_bytes = 2 * s.ck * D * (int)sizeof(T);
+  const size_t fixed = sizeof(float) * ((size_t)kMW * GP * D + 2 * (size_t)kMW * GP) +
+                       (size_t)kCW * SH::kPwBytes;
+  const size_t budget = 225 * 1024;
+  int stages = (int)((budget - fixed) / (size_t)stage_bytes);
+  stages = stages > kMaxStages ? kMaxStages : stages;
+  if (stages < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = (size_t)stages * stage_bytes + fixed;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  long long grid = sms < kGridMax ? sms : kGridMax;
+  if (grid > s.units) grid = s.units;
+  if (grid < 1) return cudaSuccess;
+  e = cudaFuncSetAttribute(decode_stream_kernel<T, D, GP>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_stream_kernel<T, D, GP><<<(unsigned)grid, kStreamThreads, smem, st>>>(
+      (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, s.ck, s.subs,
+      stages, stage_bytes, s.units, p.parts_max, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O,
+      scale * 1.4426950408889634f);
+  return cudaGetLastError();
 }
 
 template <typename T, int D>
@@ -520,28 +836,10 @@ static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const voi
       idx_out, 1.0f / sqrtf((float)D));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int nk_max = p.per_split * B;
-  const int GPv = p.G <= 4 ? 4 : 8;
-  const size_t smem2 = 2 * (size_t)nk_max * D * sizeof(T) +
-                       sizeof(float) * ((size_t)nk_max * GPv + (size_t)8 * GPv * D + 9 * GPv);
-  dim3 grid(p.splits, batch * Hkv);
-  const float sl2 = scale * 1.4426950408889634f;
-  if (p.G <= 4) {
-    e = cudaFuncSetAttribute(decode_split_kernel<T, D, 4>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
-    if (e != cudaSuccess) return e;
-    decode_split_kernel<T, D, 4><<<grid, 256, smem2, st>>>(
-        (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, p.splits,
-        p.per_split, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O, sl2);
-  } else {
-    e = cudaFuncSetAttribute(decode_split_kernel<T, D, 8>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
-    if (e != cudaSuccess) return e;
-    decode_split_kernel<T, D, 8><<<grid, 256, smem2, st>>>(
-        (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, p.splits,
-        p.per_split, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O, sl2);
-  }
-  return cudaGetLastError();
+  return p.G <= 4 ? launch_stream<T, D, 4>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale, O,
+                                           ws_idx, ws_cnt, ws_ctr, ws_part, st)
+                  : launch_stream<T, D, 8>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale, O,
+                                           ws_idx, ws_cnt, ws_ctr, ws_part, st);
 }
 
 cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,

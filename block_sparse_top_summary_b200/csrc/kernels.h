@@ -38,8 +38,7 @@ struct DecodePlan {
   int nblk_max;   // ceil(Lmax / B)
   int kk;         // effective top-k: min(topk, nblk_max)
   int width;      // idx row width: kk + 2
-  int splits;     // CTAs per (sequence, KV head) in the split-KV pass
-  int per_split;  // selected blocks handled by one split CTA
+  int parts_max;  // partial records per (sequence, KV head) the scratch holds
   size_t off_idx, off_cnt, off_part, off_ctr, bytes;
 };
 

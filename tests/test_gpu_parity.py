@@ -195,6 +195,13 @@ def test_poisoned_unselected_and_future_keys_do_not_change_output(ssa, dtype):
     (4, 16, 4, 128 * 30, 128, 128, 5, "bf16", [128 * 30, 1, 128, 129]),
     (2, 8, 1, 64 * 50, 128, 64, 1 << 30, "bf16", [64 * 50, 64 * 7 + 3]),   # all blocks
     (2, 6, 2, 16 * 200, 64, 16, 12, "bf16", [16 * 200, 16 * 77 + 5]),      # G = 3, B = 16
+    # f32, d = 128: a block is two units of 32 keys; a last block of 40 keys
+    # has a short second unit, one of 20 keys an empty one
+    (3, 8, 2, 64 * 30, 128, 64, 5, "f32", [64 * 30, 64 * 23 + 40, 64 * 12 + 20]),
+    # 64 (sequence, KV head) pairs x 18 blocks over one CTA per SM: every
+    # pair is shared by several CTAs (partial records + combine)
+    (8, 16, 8, 64 * 64, 128, 64, 16, "bf16",
+     [64 * 64, 64 * 63 + 1, 64 * 40 + 17, 64 * 64 - 5, 64 * 20, 64 * 33 + 60, 64 * 50 + 2, 64 * 17]),
 ])
 def test_decode_parity(ssa, batch, Hq, Hkv, Lmax, d, B, topk, dtype, seqlens):
     q, Kc, Vc, L = planted_decode(batch, Hq, Hkv, Lmax, d, B, clusters=5, seed=8, dtype=dtype,

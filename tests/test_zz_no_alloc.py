@@ -51,12 +51,12 @@ def test_noalloc_rejects_sizes_beyond_its_array():
     import block_sparse_top_summary_b200 as ssa
     lib = ssa.load_library()
     fake = ctypes.c_void_p(0x100000)  # never dereferenced: the size check fails first
-    need = ssa.ssa_decode_workspace_size(512, 32, 8, 65536, 128, 64, 32)
+    need = ssa.ssa_decode_workspace_size(2048, 32, 8, 65536, 128, 64, 32)
     assert need > (40 << 20)
     fn = lib.ssa_decode_noalloc
     vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     fn.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp]
     fn.restype = i
-    r = fn(fake, fake, fake, 1, fake, fake, 512, 32, 8, 65536, 128, 64, 32,
+    r = fn(fake, fake, fake, 1, fake, fake, 2048, 32, 8, 65536, 128, 64, 32,
            ctypes.c_float(0.088), fake, None, None)
     assert r == 2  # SSA_ERR_UNSUPPORTED
