@@ -32,12 +32,11 @@
 // issued and frees its TMEM.
 #include <cuda.h>
 
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 #include "ssa_debug.h"
+#include "tmap.h"
 
 namespace ssa {
 
@@ -55,13 +54,15 @@ constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s per wait
 
 
 struct __align__(8) Shared {
-  uint64_t q_full;
+  uint64_t q_full;           // Q of the current work item has landed
+  uint64_t q_empty;          // every S of the previous work item has completed
   uint64_t k_full[kNS];
   uint64_t v_full[kNS];
   uint64_t kv_empty[kNS];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done[2];
+  uint64_t o_free[2];   // per tile: the epilogue has read O (256 arrivals)
   uint64_t drain;
   uint64_t mx_full[2];  // per tile: both half-row maxima of the chunk are written
   uint64_t l_full[2];   // per tile: both half-row sums are written (epilogue)
@@ -69,7 +70,6 @@ struct __align__(8) Shared {
   float lx[2][2][128];     // [tile][half][row]
   uint32_t tmem_base;
   int abort;
-  int sel[1];  // selection of this work item (cnt entries)
 };
 
 __device__ __forceinline__ unsigned long long globaltimer() {
@@ -206,12 +206,41 @@ __device__ __forceinline__ void exp_pack32(const uint32_t (&v)[32], uint32_t (&w
 
 }  // namespace
 
+// Work item w (heaviest first: query block i = nq - 1 - w / (subs * nbg)).
+struct Item {
+  int b, g, i, h0, bg;
+};
+
+__device__ __forceinline__ Item item_of(int w, int subs, int nbg, int Hkv, int G, int nq, int HPI) {
+  Item it;
+  const int per_i = subs * nbg;
+  it.i = nq - 1 - w / per_i;
+  const int rem = w - (w / per_i) * per_i;
+  it.bg = rem / subs;
+  const int sub = rem - it.bg * subs;
+  it.b = it.bg / Hkv;
+  it.g = it.bg - it.b * Hkv;
+  it.h0 = it.g * G + sub * HPI;
+  return it;
+}
+
+template <int B>
+__device__ __forceinline__ int chunks_of(int ns) {
+  return ns <= 0 ? 0 : (B == 64) ? (ns + 1) / 2 : ns;
+}
+
+// Persistent kernel: CTA x runs work items x, x + gridDim.x, ...  Every
+// per-chunk mbarrier phase is counted by the CTA's running chunk index, so
+// the pipeline flows from one item into the next: Q of the next item loads
+// once the last S of the current one completes, its first S runs while the
+// current item's epilogue reads O, and its first P.V waits only for that
+// epilogue (o_free).
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
-    int Hq, int Hkv, int N, int nq, int max_sel, float scale_log2) {
+    int Hq, int Hkv, int N, int nq, int nbg, int max_sel, float scale_log2) {
   constexpr int HPT = 128 / B;      // query heads per M-tile
   constexpr int HPI = 2 * HPT;      // query heads per work item
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -224,22 +253,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
 
   const int G = Hq / Hkv;
   const int subs = G / HPI;
-  const int bg = blockIdx.y;
-  const int b = bg / Hkv;
-  const int g = bg - b * Hkv;
-  const int i = nq - 1 - (int)(blockIdx.x / subs);
-  const int sub = blockIdx.x % subs;
-  const int h0 = g * G + sub * HPI;  // first query head of this work item
+  const int W = nq * subs * nbg;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ns = cnt[(int64_t)bg * nq + i];
-  // cnt >= 1 for any routing output (block 0 is always selected); a zero
-  // count makes the CTA skip all work and leave its rows unwritten.
-  const int nch = ns <= 0 ? 0 : (B == 64) ? (ns + 1) / 2 : ns;
   volatile int* abort = &sh->abort;
+  auto ns_of = [&](int w) -> int {
+    if (w >= W) return 0;
+    const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI);
+    return cnt[(int64_t)it.bg * nq + it.i];
+  };
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&sh->q_full, 1);
+    ptx::mbar_init(&sh->q_empty, 1);
     for (int s = 0; s < kNS; ++s) {
       ptx::mbar_init(&sh->k_full[s], 1);
       ptx::mbar_init(&sh->v_full[s], 1);
@@ -249,17 +275,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       ptx::mbar_init(&sh->s_full[t], 1);
       ptx::mbar_init(&sh->p_full[t], 256);
       ptx::mbar_init(&sh->o_done[t], 1);
-    }
-    ptx::mbar_init(&sh->drain, 1);
-    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(&sh->o_free[t], 256);
       ptx::mbar_init(&sh->mx_full[t], 256);
       ptx::mbar_init(&sh->l_full[t], 256);
     }
+    ptx::mbar_init(&sh->drain, 1);
     sh->abort = 0;
     ptx::fence_mbar_init();
   }
-  for (int s = threadIdx.x; s < ns; s += kThreads)
-    sh->sel[s] = idx[((int64_t)bg * nq + i) * max_sel + s];
   if (warp == 1) {
     ptx::tmem_alloc(&sh->tmem_base, kTmemCols);
     ptx::tmem_relinquish();
@@ -270,55 +293,77 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   const uint32_t tmem = sh->tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && nch > 0) {
+    // ------------------------------------------------------------ producer (whole warp)
+    if (lane == 0) {
       ptx::prefetch_tmap(&tmQ);
       ptx::prefetch_tmap(&tmK);
       ptx::prefetch_tmap(&tmV);
-      ptx::mbar_arrive_expect_tx(&sh->q_full, kQBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int hh = 0; hh < HPT; ++hh)
-          for (int rg = 0; rg < B / 64; ++rg)
-            for (int c = 0; c < 2; ++c)
-              ptx::tma_load_3d(Qs + t * 32768 + c * 16384 + (hh * B + rg * 64) * 128, &tmQ,
-                               c * 64, i * B + rg * 64, b * Hq + h0 + t * HPT + hh, &sh->q_full);
-      int issued = 0;
-      for (int c = 0; c < nch; ++c) {
-        const int s = c % kNS;
-        if (c >= kNS && !wait_bar(&sh->kv_empty[s], ((c / kNS) - 1) & 1, abort)) break;
-        int y[2];
-        for (int kg = 0; kg < 2; ++kg) {
+    }
+    int gc = 0, kq = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < W; w += gridDim.x) {
+      const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI);
+      const int ns = cnt[(int64_t)it.bg * nq + it.i];
+      const int nch = chunks_of<B>(ns);
+      if (nch == 0) continue;
+      const int32_t* row = idx + ((int64_t)it.bg * nq + it.i) * max_sel;
+      int sbase = 0;
+      int selv = lane < ns ? row[lane] : 0;  // lane p holds entry sbase + p
+      // Q of this item once the previous item's S MMAs are done with Q
+      if (kq > 0 && !(ok = warp_wait_bar(&sh->q_empty, (kq - 1) & 1, abort))) break;
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(&sh->q_full, kQBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int hh = 0; hh < HPT; ++hh)
+            for (int rg = 0; rg < B / 64; ++rg)
+              for (int c = 0; c < 2; ++c)
+                ptx::tma_load_3d(Qs + t * 32768 + c * 16384 + (hh * B + rg * 64) * 128, &tmQ,
+                                 c * 64, it.i * B + rg * 64, it.b * Hq + it.h0 + t * HPT + hh,
+                                 &sh->q_full);
+      }
+      ++kq;
+      for (int c = 0; c < nch; ++c, ++gc) {
+        const int s = gc % kNS;
+        if (gc >= kNS && !(ok = warp_wait_bar(&sh->kv_empty[s], ((gc / kNS) - 1) & 1, abort))) break;
+        const int p0 = (B == 64) ? 2 * c : c;  // first selection entry of the chunk
+        if (p0 >= sbase + 32) {                // next 32 entries (p0 - sbase is even for B = 64)
+          sbase += 32;
+          selv = sbase + lane < ns ? row[sbase + lane] : 0;
+        }
+        const int j0 = __shfl_sync(0xffffffffu, selv, p0 - sbase);
+        const int j1 = (B == 64) ? __shfl_sync(0xffffffffu, selv, p0 + 1 - sbase) : 0;
+        if (lane == 0) {
+          int y[2];
           if (B == 64) {
-            const int p = 2 * c + kg;
-            y[kg] = p < ns ? sh->sel[p] * 64 : nq * B;  // past the end: zero box
+            y[0] = j0 * 64;
+            y[1] = p0 + 1 < ns ? j1 * 64 : nq * B;  // past the end: zero box
           } else {
-            y[kg] = sh->sel[c] * 128 + kg * 64;
+            y[0] = j0 * 128;
+            y[1] = j0 * 128 + 64;
           }
+          ptx::mbar_arrive_expect_tx(&sh->k_full[s], kKVBytes);
+          for (int kg = 0; kg < 2; ++kg)
+            for (int cc = 0; cc < 2; ++cc)
+              ptx::tma_load_3d(Ks + s * kKVBytes + cc * 16384 + kg * 8192, &tmK, cc * 64, y[kg],
+                               it.b * Hkv + it.g, &sh->k_full[s]);
+          ptx::mbar_arrive_expect_tx(&sh->v_full[s], kKVBytes);
+          for (int kg = 0; kg < 2; ++kg)
+            for (int cc = 0; cc < 2; ++cc)
+              ptx::tma_load_3d(Vs + s * kKVBytes + cc * 16384 + kg * 8192, &tmV, cc * 64, y[kg],
+                               it.b * Hkv + it.g, &sh->v_full[s]);
         }
-        ptx::mbar_arrive_expect_tx(&sh->k_full[s], kKVBytes);
-        for (int kg = 0; kg < 2; ++kg)
-          for (int cc = 0; cc < 2; ++cc)
-            ptx::tma_load_3d(Ks + s * kKVBytes + cc * 16384 + kg * 8192, &tmK, cc * 64, y[kg],
-                             b * Hkv + g, &sh->k_full[s]);
-        ptx::mbar_arrive_expect_tx(&sh->v_full[s], kKVBytes);
-        for (int kg = 0; kg < 2; ++kg)
-          for (int cc = 0; cc < 2; ++cc)
-            ptx::tma_load_3d(Vs + s * kKVBytes + cc * 16384 + kg * 8192, &tmV, cc * 64, y[kg],
-                             b * Hkv + g, &sh->v_full[s]);
-        issued = c + 1;
       }
-      if (*abort) {
-        // let every issued copy land before the CTA's shared memory goes away
-        for (int c = (issued > kNS ? issued - kNS : 0); c < issued; ++c) {
-          const int s = c % kNS;
-          const uint32_t ph = (c / kNS) & 1;
-          volatile int no_abort = 0;
-          wait_bar(&sh->k_full[s], ph, &no_abort);
-          wait_bar(&sh->v_full[s], ph, &no_abort);
-        }
-        volatile int no_abort = 0;
-        wait_bar(&sh->q_full, 0, &no_abort);
+    }
+    if (!ok && lane == 0) {
+      // let every issued copy land before the CTA's shared memory goes away
+      volatile int no_abort = 0;
+      for (int c = (gc > kNS ? gc - kNS : 0); c < gc; ++c) {
+        const int s = c % kNS;
+        const uint32_t ph = (c / kNS) & 1;
+        wait_bar(&sh->k_full[s], ph, &no_abort);
+        wait_bar(&sh->v_full[s], ph, &no_abort);
       }
+      if (kq > 0) wait_bar(&sh->q_full, (kq - 1) & 1, &no_abort);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -326,8 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       const uint32_t qa = ptx::smem_u32(Qs);
       const uint32_t ka = ptx::smem_u32(Ks);
       const uint32_t va = ptx::smem_u32(Vs);
-      bool ok = nch > 0 && wait_bar(&sh->q_full, 0, abort) && wait_bar(&sh->k_full[0], 0, abort);
-      bool any = false;
+      bool any = false, ok = true;
       auto issue_qk = [&](int t, int s) {
         ptx::tc_fence_after();
         for (int kk = 0; kk < 8; ++kk) {
@@ -345,27 +389,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
                       (c > 0 || kk > 0) ? 1u : 0u);
         ptx::mma_commit(&sh->o_done[t]);
       };
-      if (ok) {
-        issue_qk(0, 0);
-        issue_qk(1, 0);
+      int gc = 0, kq = 0;
+      int ns_next = ns_of(blockIdx.x);
+      for (int w = blockIdx.x; ok && w < W; w += gridDim.x) {
+        const int ns = ns_next;
+        ns_next = ns_of(w + gridDim.x);
+        const int nch = chunks_of<B>(ns);
+        if (nch == 0) continue;
+        if (!(ok = wait_bar(&sh->q_full, kq & 1, abort))) break;
+        if (!(ok = wait_bar(&sh->k_full[gc % kNS], (gc / kNS) & 1, abort))) break;
+        // S of the new item overwrites P of the previous one: issued after
+        // its P.V, and tcgen05 MMAs of one thread run in issue order
+        issue_qk(0, gc % kNS);
+        issue_qk(1, gc % kNS);
         any = true;
-      }
-      for (int c = 0; ok && c < nch; ++c) {
-        const int s = c % kNS;
-        const uint32_t ph = (c / kNS) & 1;
-        if (!(ok = wait_bar(&sh->v_full[s], ph, abort))) break;
-        if (!(ok = wait_bar(&sh->p_full[0], c & 1, abort))) break;
-        issue_pv(0, s, c);
-        const bool more = c + 1 < nch;
-        const int s1 = (c + 1) % kNS;
-        if (more) {
-          if (!(ok = wait_bar(&sh->k_full[s1], ((c + 1) / kNS) & 1, abort))) break;
-          issue_qk(0, s1);
+        if (nch == 1) ptx::mma_commit(&sh->q_empty);
+        for (int c = 0; c < nch; ++c) {
+          const int g = gc + c;
+          const int s = g % kNS;
+          if (!(ok = wait_bar(&sh->v_full[s], (g / kNS) & 1, abort))) break;
+          if (!(ok = wait_bar(&sh->p_full[0], g & 1, abort))) break;
+          if (c == 0 && kq > 0 && !(ok = wait_bar(&sh->o_free[0], (kq - 1) & 1, abort))) break;
+          issue_pv(0, s, c);
+          const bool more = c + 1 < nch;
+          const int s1 = (g + 1) % kNS;
+          if (more) {
+            if (!(ok = wait_bar(&sh->k_full[s1], ((g + 1) / kNS) & 1, abort))) break;
+            issue_qk(0, s1);
+          }
+          if (!(ok = wait_bar(&sh->p_full[1], g & 1, abort))) break;
+          if (c == 0 && kq > 0 && !(ok = wait_bar(&sh->o_free[1], (kq - 1) & 1, abort))) break;
+          issue_pv(1, s, c);
+          ptx::mma_commit(&sh->kv_empty[s]);
+          if (more) {
+            issue_qk(1, s1);
+            if (c + 2 == nch) ptx::mma_commit(&sh->q_empty);  // last S of the item issued
+          }
         }
-        if (!(ok = wait_bar(&sh->p_full[1], c & 1, abort))) break;
-        issue_pv(1, s, c);
-        ptx::mma_commit(&sh->kv_empty[s]);
-        if (more) issue_qk(1, s1);
+        gc += nch;
+        ++kq;
       }
       if (any) {
         // every MMA issued by this thread has completed once `drain` flips
@@ -380,156 +442,176 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const int half = ((warp - 2) >> 2) & 1; // key half of the chunk: columns 64 half ..
     const int quarter = warp & 3;           // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;      // row in the tile = TMEM lane
-    const int hh = r / B;
-    const int pos = i * B + (r % B);
-    const int h = h0 + t * HPT + hh;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128 + half * 64;
     const uint32_t tO = tmem + lane_off + 256 + t * 128 + half * 64;
-    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int c = 0; c < nch; ++c) {
-      if (!(ok = warp_wait_bar(&sh->s_full[t], c & 1, abort))) break;
-      ptx::tc_fence_after();
-      const bool last = (c == nch - 1);
-      // causal mask / missing block, only in the chunk holding the diagonal:
-      // key column n (0..127) of block half kg is valid iff (n mod 64) <=
-      // lim[kg] (B = 64), or n <= lim[0] (B = 128)
-      int lim[2] = {127, 127};
-      if (last) {
-        if (B == 64) {
-          for (int kg = 0; kg < 2; ++kg) {
-            const int p = 2 * c + kg;
-            const int j = p < ns ? sh->sel[p] : -1;
-            lim[kg] = j < 0 ? -1 : (j == i ? (r & 63) : 63);
+    int gc = 0, kq = 0;
+    int ns_next = ns_of(blockIdx.x);
+    for (int w = blockIdx.x; ok && w < W; w += gridDim.x) {
+      const int ns = ns_next;
+      ns_next = ns_of(w + gridDim.x);
+      const int nch = chunks_of<B>(ns);
+      if (nch == 0) continue;
+      const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI);
+      const int hh = r / B;
+      const int pos = it.i * B + (r % B);
+      const int h = it.h0 + t * HPT + hh;
+      float m_used = -INFINITY, l = 0.f;
+      for (int c = 0; c < nch; ++c) {
+        const int g = gc + c;
+        if (!(ok = warp_wait_bar(&sh->s_full[t], g & 1, abort))) break;
+        ptx::tc_fence_after();
+        const bool last = (c == nch - 1);
+        // causal mask / missing block, only in the chunk holding the diagonal.
+        // Selections are ascending and end with the diagonal block, so the
+        // last chunk is (diagonal, missing) when ns is odd and (full,
+        // diagonal) when it is even (B = 64), or the diagonal (B = 128).
+        // Key column n (0..127) of block half kg is valid iff (n mod 64) <=
+        // lim[kg] (B = 64), or n <= lim[0] (B = 128).
+        int lim[2] = {127, 127};
+        if (last) {
+          if (B == 64) {
+            if (ns & 1) {
+              lim[0] = r & 63;
+              lim[1] = -1;
+            } else {
+              lim[0] = 63;
+              lim[1] = r & 63;
+            }
+          } else {
+            lim[0] = lim[1] = r;
           }
-        } else {
-          lim[0] = lim[1] = (sh->sel[c] == i) ? r : 127;
         }
-      }
-      // pass 1: this half's maximum, then the other half's through shared memory
-      float pm = -INFINITY;
+        // pass 1: this half's maximum, then the other half's through shared memory
+        float pm = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t v[32];
-        ptx::tmem_ld32(tS + q * 32, v);
-        ptx::tmem_wait_ld();
-        if (last) mask32<B>(v, half * 64 + q * 32, lim);
-        pm = max32(v, pm);
-      }
-      sh->mx[c & 1][t][half][r] = pm;
-      ptx::mbar_arrive(&sh->mx_full[t]);
-      // The two halves of a row must use one reference max.  From chunk 1 on,
-      // P is computed optimistically with the current reference m_used while
-      // the other half's maximum is in flight; the pass is redone only if the
-      // row max exceeds m_used by more than 2^kSlack (then P, l and O would
-      // leave a comfortable fp32 / bf16 range).  Chunk 0 waits for the
-      // exchange first.
-      constexpr float kSlack = 64.0f;
-      float rmax = -INFINITY;
-      bool have_rmax = false;
-      if (c == 0) {
-        if (!(ok = warp_wait_bar(&sh->mx_full[t], c & 1, abort))) break;
-        rmax = fmaxf(pm, sh->mx[c & 1][t][half ^ 1][r]) * scale_log2;
-        m_used = rmax;
-        have_rmax = true;
-      }
-      bool need = false;
-      float alpha = 1.0f;
-      uint64_t acc = 0;
-      uint32_t w0[16], w1[16];  // P of this half, stored only once it is final
-      for (int attempt = 0; attempt < 2; ++attempt) {
-        const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-        const uint64_t s2 = pack2(scale_log2, scale_log2);
-        const uint64_t c2 = pack2(-mu, -mu);
-        // pass 2: p = 2^(s*scale - m) as bf16 pairs (S stays intact until the
-        // pairs are stored, so a redo can read it again)
-        acc = 0;
-        {
+        for (int q = 0; q < 2; ++q) {
           uint32_t v[32];
-          ptx::tmem_ld32(tS, v);
+          ptx::tmem_ld32(tS + q * 32, v);
           ptx::tmem_wait_ld();
-          if (last) mask32<B>(v, half * 64, lim);
-          exp_pack32(v, w0, s2, c2, acc);
-          ptx::tmem_ld32(tS + 32, v);
-          ptx::tmem_wait_ld();
-          if (last) mask32<B>(v, half * 64 + 32, lim);
-          exp_pack32(v, w1, s2, c2, acc);
+          if (last) mask32<B>(v, half * 64 + q * 32, lim);
+          pm = max32(v, pm);
         }
-        if (!have_rmax) {
-          if (!(ok = warp_wait_bar(&sh->mx_full[t], c & 1, abort))) break;
-          rmax = fmaxf(pm, sh->mx[c & 1][t][half ^ 1][r]) * scale_log2;
+        sh->mx[g & 1][t][half][r] = pm;
+        ptx::mbar_arrive(&sh->mx_full[t]);
+        // The two halves of a row must use one reference max.  From chunk 1
+        // on, P is computed optimistically with the current reference m_used
+        // while the other half's maximum is in flight; the pass is redone only
+        // if the row max exceeds m_used by more than 2^kSlack (then P, l and O
+        // would leave a comfortable fp32 / bf16 range).  Chunk 0 waits for the
+        // exchange first.
+        constexpr float kSlack = 64.0f;
+        float rmax = -INFINITY;
+        bool have_rmax = false;
+        if (c == 0) {
+          if (!(ok = warp_wait_bar(&sh->mx_full[t], g & 1, abort))) break;
+          rmax = fmaxf(pm, sh->mx[g & 1][t][half ^ 1][r]) * scale_log2;
+          m_used = rmax;
           have_rmax = true;
         }
-        // both halves of a row see the same rmax and m_used, so they decide
-        // alike; the redo itself is warp-uniform (the loads and shuffles it
-        // runs are warp-collective), rows that do not need it recompute the
-        // same values
-        const bool my_need = attempt == 0 && c > 0 && rmax > m_used + kSlack;
-        if (my_need) {
-          need = true;
-          alpha = ex2_mufu(m_used - rmax);
-          l *= alpha;
-          m_used = rmax;
+        bool need = false;
+        float alpha = 1.0f;
+        uint64_t acc = 0;
+        uint32_t w0[16], w1[16];  // P of this half, stored only once it is final
+        for (int attempt = 0; attempt < 2; ++attempt) {
+          const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+          const uint64_t s2 = pack2(scale_log2, scale_log2);
+          const uint64_t c2 = pack2(-mu, -mu);
+          // pass 2: p = 2^(s*scale - m) as bf16 pairs (S stays intact until
+          // the pairs are stored, so a redo can read it again)
+          acc = 0;
+          {
+            uint32_t v[32];
+            ptx::tmem_ld32(tS, v);
+            ptx::tmem_wait_ld();
+            if (last) mask32<B>(v, half * 64, lim);
+            exp_pack32(v, w0, s2, c2, acc);
+            ptx::tmem_ld32(tS + 32, v);
+            ptx::tmem_wait_ld();
+            if (last) mask32<B>(v, half * 64 + 32, lim);
+            exp_pack32(v, w1, s2, c2, acc);
+          }
+          if (!have_rmax) {
+            if (!(ok = warp_wait_bar(&sh->mx_full[t], g & 1, abort))) break;
+            rmax = fmaxf(pm, sh->mx[g & 1][t][half ^ 1][r]) * scale_log2;
+            have_rmax = true;
+          }
+          // both halves of a row see the same rmax and m_used, so they decide
+          // alike; the redo itself is warp-uniform (the loads and shuffles it
+          // runs are warp-collective), rows that do not need it recompute the
+          // same values
+          const bool my_need = attempt == 0 && c > 0 && rmax > m_used + kSlack;
+          if (my_need) {
+            need = true;
+            alpha = ex2_mufu(m_used - rmax);
+            l *= alpha;
+            m_used = rmax;
+          }
+          if (__any_sync(0xffffffffu, my_need)) continue;  // redo pass 2
+          break;
         }
-        if (__any_sync(0xffffffffu, my_need)) continue;  // redo pass 2
-        break;
-      }
-      if (!ok) break;
-      // P words land on this half's first 32 S columns, all consumed by now
-      ptx::tmem_st16(tS, w0);
-      ptx::tmem_st16(tS + 16, w1);
-      if (!ok) break;
-      l += sum2(acc);
-      if (__any_sync(0xffffffffu, need)) {
-        // O must hold PV of the previous chunk before it is rescaled; PV of
-        // this chunk is not issued before this thread arrives on p_full.
-        if (!(ok = warp_wait_bar(&sh->o_done[t], (c - 1) & 1, abort))) break;
-        ptx::tc_fence_after();
+        if (!ok) break;
+        // P words land on this half's first 32 S columns, all consumed by now
+        ptx::tmem_st16(tS, w0);
+        ptx::tmem_st16(tS + 16, w1);
+        l += sum2(acc);
+        if (__any_sync(0xffffffffu, need)) {
+          // O must hold P.V of the previous chunk before it is rescaled (S of
+          // this chunk was issued after it); P.V of this chunk is not issued
+          // before this thread arrives on p_full.
+          if (!(ok = warp_wait_bar(&sh->o_done[t], (g - 1) & 1, abort))) break;
+          ptx::tc_fence_after();
 #pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
-          uint32_t ov[32];
-          ptx::tmem_ld32(tO + q * 32, ov);
-          ptx::tmem_wait_ld();
+          for (int q = 0; q < 2; ++q) {
+            uint32_t ov[32];
+            ptx::tmem_ld32(tO + q * 32, ov);
+            ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          ptx::tmem_st32(tO + q * 32, ov);
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            ptx::tmem_st32(tO + q * 32, ov);
+          }
         }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&sh->p_full[t]);
       }
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&sh->p_full[t]);
-    }
-    // ------------------------------------------------------------ epilogue
-    if (ok && nch > 0) {
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
       sh->lx[t][half][r] = l;
       ptx::mbar_arrive(&sh->l_full[t]);
-      ok = warp_wait_bar(&sh->l_full[t], 0, abort);
-    }
-    if (ok && nch > 0 && warp_wait_bar(&sh->o_done[t], (nch - 1) & 1, abort)) {
+      if (!(ok = warp_wait_bar(&sh->l_full[t], kq & 1, abort))) break;
+      // S of the item's last chunk was issued after the P.V before it, so
+      // o_done is at the phase of the last P.V or past it: one parity wait.
+      if (!(ok = warp_wait_bar(&sh->o_done[t], (gc + nch - 1) & 1, abort))) break;
       ptx::tc_fence_after();
       const float lrow = sh->lx[t][0][r] + sh->lx[t][1][r];
       const float inv = 1.0f / lrow;
       const bool store = pos < N;
-      __nv_bfloat16* orow = O + (((int64_t)b * Hq + h) * N + (store ? pos : 0)) * 128 + half * 64;
+      __nv_bfloat16* orow = O + (((int64_t)it.b * Hq + h) * N + (store ? pos : 0)) * 128 + half * 64;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         uint32_t ov[32];
         ptx::tmem_ld32(tO + q * 32, ov);
         ptx::tmem_wait_ld();
-        uint32_t w[16];
+        uint32_t wv[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          w[e] = cvt_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+          wv[e] = cvt_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
         }
       }
+      // O of this tile is read: the next item's first P.V may overwrite it
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&sh->o_free[t]);
       if (store && half == 0 && lse != nullptr)
-        lse[((int64_t)b * Hq + h) * N + pos] = (m_used + log2f(lrow)) * 0.69314718055994530942f;
+        lse[((int64_t)it.b * Hq + h) * N + pos] = (m_used + log2f(lrow)) * 0.69314718055994530942f;
+      gc += nch;
+      ++kq;
     }
   }
   ptx::tc_fence_before();
@@ -557,56 +639,31 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns) {
 // ---------------------------------------------------------------- host side
 namespace {
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// [heads, rows, 128] bf16 viewed as a 3-D tensor (d, rows, heads); 64 x 64 boxes.
-bool make_map(CUtensorMap* m, const void* ptr, int rows, int heads) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)rows * 128 * 2};
-  cuuint32_t box[3] = {64, 64, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int B>
 cudaError_t launch_tc_t(const void* Q, const void* K, const void* V, const int32_t* idx,
                         const int32_t* cnt, int batch, int Hq, int Hkv, int N, int max_sel,
                         float scale, void* O, float* lse, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, N, batch * Hq) || !make_map(&mk, K, N, batch * Hkv) ||
-      !make_map(&mv, V, N, batch * Hkv))
+  if (!make_bf16_map(&mq, Q, 128, N, batch * Hq, 64) ||
+      !make_bf16_map(&mk, K, 128, N, batch * Hkv, 64) ||
+      !make_bf16_map(&mv, V, 128, N, batch * Hkv, 64))
     return cudaErrorInvalidValue;
   const int nq = (N + B - 1) / B;
   const int G = Hq / Hkv;
   const int subs = G / (2 * (128 / B));
-  const size_t smem = 1024 + kSmemBytes + sizeof(Shared) + sizeof(int) * (size_t)max_sel;
+  const long long items = (long long)nq * subs * batch * Hkv;
+  if (items <= 0) return cudaSuccess;
+  if (items > (1ll << 30)) return cudaErrorInvalidValue;
+  const size_t smem = 1024 + kSmemBytes + sizeof(Shared);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(nq * subs, batch * Hkv);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = (int)(items < sms ? items : sms);  // one persistent CTA per SM
   attn_tc_kernel<B><<<grid, kThreads, smem, st>>>(mq, mk, mv, idx, cnt, (__nv_bfloat16*)O, lse,
-                                                  Hq, Hkv, N, nq, max_sel,
+                                                  Hq, Hkv, N, nq, batch * Hkv, max_sel,
                                                   scale * 1.4426950408889634f);
   return cudaGetLastError();
 }
