@@ -13,16 +13,20 @@
 //   2. split-KV attention, a persistent streaming kernel (one CTA per SM).
 //      The selected blocks of all (sequence, KV head) pairs are cut into
 //      units of at most 32 KB of K + V rows; each CTA owns an equal
-//      contiguous run of units.  A producer warp fetches each unit's K rows
-//      and V rows (contiguous in the BHND cache) with one untiled bulk copy
-//      each into a ring of shared stages; sixteen consumer warps split every
-//      unit's keys and keep their own online softmax (max m, sum l,
-//      unnormalised o).  Where the run leaves a (sequence, KV head) the warps
-//      are merged; a pair split between CTAs is finished by the last of them
-//      (atomic counter) with a log-sum-exp combine of the partial records.
+//      contiguous run of units.  A producer warp copies each unit into a
+//      ring of shared stages.  bf16: one TMA tensor box per 64 columns
+//      (128-byte swizzle), and each of four consumer warps takes whole units
+//      on mma.sync tensor-core tiles (the group's heads are the rows).  fp32:
+//      one untiled bulk copy each for the K rows and the V rows, and sixteen
+//      consumer warps split every unit's keys in fp32 FMA.  Every consumer
+//      warp keeps its own online softmax (max m, sum l, unnormalised o).
+//      Where the run leaves a (sequence, KV head) the warps are merged; a
+//      pair split between CTAs is finished by the last of them (atomic
+//      counter) with a log-sum-exp combine of the partial records.
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "tmap.h"
 
 namespace ssa {
 
@@ -317,6 +321,10 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
 }
 
+__device__ __forceinline__ void mma_consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(4 * 32) : "memory");
+}
+
 template <int VB>
 __device__ __forceinline__ void ld_vec(const void* p, uint32_t (&w)[VB / 4]) {
   if constexpr (VB == 16) {
@@ -369,7 +377,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
     const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
     float* __restrict__ ws_part, int* __restrict__ ws_ctr, T* __restrict__ O, float scale_log2) {
   using SH = StreamShape<T, D, GP>;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ int info[kMaxStages];  // rows held by each stage
   __shared__ int s_abort, s_last;
@@ -733,6 +741,362 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
   }
 }
 
+// ------------------------------------------------- 2b. split-KV attention, bf16
+// The same unit stream as decode_stream_kernel, with the two contractions of
+// a unit on mma.sync tensor-core tiles (m16n8k16, bf16 in, fp32 accumulate):
+//   S = Qg . K^T  (rows: the G <= 8 query heads of the group, rows 8-15 zero)
+//   O += P . V    (P rounded to bf16, as in the prefill kernel)
+// A unit's K and V rows arrive as 64-column boxes with the 128-byte swizzle
+// (TMA tensor copies), so the ldmatrix row reads are conflict-free.  One
+// consumer warp takes a whole unit (units n = warp mod kMmaCW) and keeps its
+// own online softmax; P.V reuses the S accumulators as A fragments directly.
+namespace {
+
+constexpr int kMmaCW = 4;                          // consumer warps
+constexpr int kMmaThreads = 32 * (kMmaCW + 1);     // + one producer warp
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// d += A . B for one m16n8k16 tile with A rows 8-15 zero (a1 = a3 = 0).
+__device__ __forceinline__ void mma_rows8(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ seqlens, int Hq, int Hkv,
+    int Lmax, int B, int width, int CK, int subs, int stages, long long U, int parts_max,
+    const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
+    float* __restrict__ ws_part, int* __restrict__ ws_ctr, __nv_bfloat16* __restrict__ O,
+    float scale_log2) {
+  constexpr int CKM = 32768 / (4 * D);  // most keys per unit (32 KB of K + V)
+  constexpr int NT = CKM / 8;           // S column tiles
+  constexpr int KS = D / 16;            // k steps of S
+  constexpr int ON = D / 8;             // O column tiles
+  constexpr int NB = D / 64;            // 64-column boxes per row block
+  constexpr float kLazy = 8.0f;         // rescale O only when the max grows by more (log2)
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
+  __shared__ int info[kMaxStages];
+  __shared__ int s_abort, s_last;
+
+  const int G = Hq / Hkv;
+  const int Ubg = width * subs;
+  const int tile_bytes = CK * D * 2;  // K (or V) rows of one unit
+  const int stage_bytes = 2 * tile_bytes;
+  const long long grid = gridDim.x;
+  const long long u0 = (long long)blockIdx.x * U / grid;
+  const long long u1 = ((long long)blockIdx.x + 1) * U / grid;
+  const int nunits = (int)(u1 - u0);
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  volatile int* abort = &s_abort;
+  float* ow = reinterpret_cast<float*>(base + (size_t)stages * stage_bytes);  // [kMmaCW][8][D]
+  float* mw = ow + kMmaCW * 8 * D;                                              // [kMmaCW][8]
+  float* lw = mw + kMmaCW * 8;                                                  // [kMmaCW][8]
+
+  if (t == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    s_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kMmaCW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmK);
+      ptx::prefetch_tmap(&tmV);
+    }
+    auto resolve = [&](long long u, int& y, int& rows) {
+      y = 0;
+      rows = 0;
+      if (u >= u1) return;
+      const int bg = (int)(u / Ubg);
+      const int rem = (int)(u - (long long)bg * Ubg);
+      const int s = rem / subs, r = rem - s * subs;
+      if (s >= ws_cnt[bg]) return;
+      const int j = ws_idx[(int64_t)bg * width + s];
+      const int L = seqlens[bg / Hkv];
+      const int k0 = j * B + r * CK;
+      const int rr = min(CK, min(L, (j + 1) * B) - k0);
+      if (rr <= 0) return;
+      rows = rr;
+      y = k0;
+    };
+    int y_n, rows_n;
+    resolve(u0 + lane, y_n, rows_n);
+    int issued = 0;
+    bool ok = true;
+    for (int b0 = 0; ok && b0 < nunits; b0 += 32) {
+      const int y_c = y_n, rows_c = rows_n;
+      resolve(u0 + b0 + 32 + lane, y_n, rows_n);
+      const int cntb = min(32, nunits - b0);
+      for (int i = 0; i < cntb; ++i) {
+        const int n = b0 + i;
+        const int st = n % stages;
+        const int y = __shfl_sync(0xffffffffu, y_c, i);
+        const int rows = __shfl_sync(0xffffffffu, rows_c, i);
+        if (n >= stages && !(ok = warp_wait_bounded(&empty[st], ((n / stages) - 1) & 1, abort)))
+          break;
+        if (lane == 0) {
+          info[st] = rows;
+          if (rows > 0) {
+            const int bg = (int)((u0 + n) / Ubg);
+            unsigned char* dst = base + (size_t)st * stage_bytes;
+            // whole boxes land (rows past the sequence are masked, rows past
+            // the cache read as zeros), so the byte count is fixed
+            ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)stage_bytes);
+            for (int bx = 0; bx < NB; ++bx) {
+              ptx::tma_load_3d(dst + bx * CK * 128, &tmK, bx * 64, y, bg, &full[st]);
+              ptx::tma_load_3d(dst + tile_bytes + bx * CK * 128, &tmV, bx * 64, y, bg, &full[st]);
+            }
+          } else {
+            ptx::mbar_arrive(&full[st]);
+          }
+        }
+        issued = n + 1;
+      }
+    }
+    // every copy issued lands before the CTA may exit (also after an abort)
+    if (lane == 0) {
+      volatile int no_abort = 0;
+      for (int n = max(0, issued - stages); n < issued; ++n)
+        wait_bounded(&full[n % stages], (uint32_t)(n / stages) & 1u, &no_abort);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int gr = lane >> 2;  // fragment row = query head of the group (valid if < G)
+  const int tq = lane & 3;
+  uint32_t qa[KS][2];        // A fragments of q: columns 16 ks + 2 tq (+8)
+  float oc[ON][4];           // O accumulators (elements 2, 3: rows 8-15, stay 0)
+  float m_run = -INFINITY, l_run = 0.f;
+  int cur = -1;
+  // ldmatrix lane roles: matrix lane >> 3, row lane & 7
+  const int lm = lane >> 3, lr = lane & 7;
+
+  for (int n = 0; n <= nunits; ++n) {
+    const int bg = n < nunits ? (int)((u0 + n) / Ubg) : -2;
+    if (bg != cur) {
+      if (cur >= 0) {
+        // ---- end of a (sequence, KV head): merge the consumer warps
+        float l = l_run;
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if (tq == 0) {
+          mw[warp * 8 + gr] = m_run;
+          lw[warp * 8 + gr] = l;
+        }
+#pragma unroll
+        for (int nt = 0; nt < ON; ++nt)
+          *reinterpret_cast<float2*>(ow + ((size_t)warp * 8 + gr) * D + nt * 8 + 2 * tq) =
+              make_float2(oc[nt][0], oc[nt][1]);
+        mma_consumer_sync();
+        const int b = cur / Hkv, g = cur - b * Hkv;
+        const long long uf = (long long)cur * Ubg;
+        const int xf = cta_of_unit(uf, U, grid);
+        const int nparts = cta_of_unit(uf + Ubg - 1, U, grid) - xf + 1;
+        float* part = ws_part + ((int64_t)cur * parts_max + (blockIdx.x - xf)) * part_floats<D>(G);
+        for (int e = t; e < G * D; e += kMmaCW * 32) {
+          const int h = e / D, dd = e - h * D;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kMmaCW; ++w) M = fmaxf(M, mw[w * 8 + h]);
+          float num = 0.f, den = 0.f;
+#pragma unroll
+          for (int w = 0; w < kMmaCW; ++w) {
+            const float mwv = mw[w * 8 + h];
+            if (mwv == -INFINITY) continue;
+            const float sc = ex2_approx(mwv - M);
+            num = fmaf(sc, ow[((size_t)w * 8 + h) * D + dd], num);
+            den = fmaf(sc, lw[w * 8 + h], den);
+          }
+          if (nparts == 1) {
+            store_out(O + ((int64_t)b * Hq + g * G + h) * D + dd, den > 0.f ? num / den : 0.f);
+          } else {
+            part[2 * G + h * D + dd] = num;
+            if (dd == 0) {
+              part[h] = M;
+              part[G + h] = den;
+            }
+          }
+        }
+        if (nparts > 1) __threadfence();
+        mma_consumer_sync();
+        if (nparts > 1) {
+          if (t == 0) s_last = (atomicAdd(&ws_ctr[cur], 1) == nparts - 1);
+          mma_consumer_sync();
+          if (s_last) {
+            __threadfence();
+            const float* parts = ws_part + (int64_t)cur * parts_max * part_floats<D>(G);
+            for (int e = t; e < G * D; e += kMmaCW * 32) {
+              const int h = e / D, dd = e - h * D;
+              float M = -INFINITY;
+              for (int p = 0; p < nparts; ++p)
+                M = fmaxf(M, __ldcg(parts + (int64_t)p * part_floats<D>(G) + h));
+              float num = 0.f, den = 0.f;
+              for (int p = 0; p < nparts; ++p) {
+                const float* pp = parts + (int64_t)p * part_floats<D>(G);
+                const float mp = __ldcg(pp + h);
+                if (mp == -INFINITY) continue;
+                const float sc = ex2_approx(mp - M);
+                den = fmaf(sc, __ldcg(pp + G + h), den);
+                num = fmaf(sc, __ldcg(pp + 2 * G + h * D + dd), num);
+              }
+              store_out(O + ((int64_t)b * Hq + g * G + h) * D + dd, den > 0.f ? num / den : 0.f);
+            }
+          }
+        }
+      }
+      if (n == nunits) break;
+      // ---- start of a (sequence, KV head): the group's query rows, fresh state
+      cur = bg;
+      {
+        const int b = bg / Hkv, g = bg - b * Hkv;
+        const bool has = gr < G;
+        const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+            q + ((int64_t)b * Hq + g * G + (has ? gr : 0)) * D + 2 * tq);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qa[ks][0] = has ? qp[ks * 8] : 0u;
+          qa[ks][1] = has ? qp[ks * 8 + 4] : 0u;
+        }
+#pragma unroll
+        for (int nt = 0; nt < ON; ++nt) oc[nt][0] = oc[nt][1] = oc[nt][2] = oc[nt][3] = 0.f;
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
+    }
+    if (n % kMmaCW != warp) continue;
+
+    // ---- one unit
+    const int st = n % stages;
+    if (warp_wait_bounded(&full[st], (uint32_t)(n / stages) & 1u, abort)) {
+      const int rows = info[st];
+      if (rows > 0) {
+        unsigned char* stg = base + (size_t)st * stage_bytes;
+        const uint32_t sK = ptx::smem_u32(stg);
+        const uint32_t sV = sK + tile_bytes;
+        const int np = CK / 16;  // 16-key groups in the unit
+        if (rows < CK) {
+          // V rows past the sequence may hold anything: make them zero so
+          // that P = 0 times them stays 0
+          for (int e = lane; e < (CK - rows) * NB * 8; e += 32) {
+            const int rr = rows + e / (NB * 8), c = e % (NB * 8);
+            *reinterpret_cast<uint4*>(stg + tile_bytes + (c >> 3) * CK * 128 + rr * 128 +
+                                      (c & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          __syncwarp();
+        }
+        // S = q . K^T
+        float sc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+        for (int p = 0; p < NT / 2; ++p) {
+          if (p < np) {
+            const int key = 16 * p + (lm >> 1) * 8 + lr;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              const int chunk = ((2 * ks) & 7) + (lm & 1);
+              const uint32_t addr = sK + (ks >> 2) * CK * 128 + key * 128 + ((chunk ^ (key & 7)) << 4);
+              uint32_t r0, r1, r2, r3;
+              ldsm_x4(addr, r0, r1, r2, r3);
+              mma_rows8(sc[2 * p], qa[ks][0], qa[ks][1], r0, r1);
+              mma_rows8(sc[2 * p + 1], qa[ks][0], qa[ks][1], r2, r3);
+            }
+          }
+        }
+        // online softmax for row gr (log2 domain); keys >= rows are masked
+        float cm = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = nt * 8 + 2 * tq + e;
+            const float x = key < rows ? sc[nt][e] * scale_log2 : -INFINITY;
+            sc[nt][e] = x;
+            cm = fmaxf(cm, x);
+          }
+        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+        if (cm > m_run + kLazy) {  // lazy: P stays below 2^kLazy otherwise
+          const float alpha = ex2_approx(m_run - cm);  // 0 on the first unit
+          l_run *= alpha;
+#pragma unroll
+          for (int nt = 0; nt < ON; ++nt) {
+            oc[nt][0] *= alpha;
+            oc[nt][1] *= alpha;
+          }
+          m_run = cm;
+        }
+        uint32_t pa[NT / 2][2];
+#pragma unroll
+        for (int p = 0; p < NT / 2; ++p) {
+          const float p0 = ex2_approx(sc[2 * p][0] - m_run), p1 = ex2_approx(sc[2 * p][1] - m_run);
+          const float p2 = ex2_approx(sc[2 * p + 1][0] - m_run);
+          const float p3 = ex2_approx(sc[2 * p + 1][1] - m_run);
+          l_run += (p0 + p1) + (p2 + p3);
+          pa[p][0] = pack_bf16x2(p0, p1);
+          pa[p][1] = pack_bf16x2(p2, p3);
+        }
+        // O += P . V
+#pragma unroll
+        for (int p = 0; p < NT / 2; ++p) {
+          if (p < np) {
+            const int key = 16 * p + (lm & 1) * 8 + lr;
+#pragma unroll
+            for (int qd = 0; qd < ON / 2; ++qd) {
+              const int chunk = 2 * qd + (lm >> 1);
+              const uint32_t addr =
+                  sV + (chunk >> 3) * CK * 128 + key * 128 + (((chunk & 7) ^ (key & 7)) << 4);
+              uint32_t r0, r1, r2, r3;
+              ldsm_x4_t(addr, r0, r1, r2, r3);
+              mma_rows8(oc[2 * qd], pa[p][0], pa[p][1], r0, r1);
+              mma_rows8(oc[2 * qd + 1], pa[p][0], pa[p][1], r2, r3);
+            }
+          }
+        }
+        if (rows < CK) ptx::fence_proxy_async_smem();  // generic zero stores before the next TMA
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[st]);
+  }
+}
+
 namespace {
 
 // Unit geometry of the streaming kernel for one element size.
@@ -816,6 +1180,41 @@ static cudaError_t launch_stream(const DecodePlan& p, const void* q, const void*
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_mma(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
+                              const int32_t* seqlens, int batch, int Hq, int Hkv, int Lmax, int B,
+                              float scale, void* O, int32_t* ws_idx, int32_t* ws_cnt, int* ws_ctr,
+                              float* ws_part, cudaStream_t st) {
+  const StreamGeom s = stream_geom(batch * Hkv, p.width, D, B, 2);
+  const int stage_bytes = 4 * s.ck * D;
+  const size_t fixed = sizeof(float) * ((size_t)kMmaCW * 8 * D + 2 * (size_t)kMmaCW * 8);
+  const size_t budget = 224 * 1024;  // dynamic shared memory, the 1 KB alignment slack included
+  int stages = (int)((budget - 1024 - fixed) / (size_t)stage_bytes);
+  stages = stages > kMaxStages ? kMaxStages : stages;
+  if (stages < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = 1024 + (size_t)stages * stage_bytes + fixed;
+  CUtensorMap mk, mv;
+  if (!make_bf16_map(&mk, Kc, D, Lmax, batch * Hkv, s.ck) ||
+      !make_bf16_map(&mv, Vc, D, Lmax, batch * Hkv, s.ck))
+    return cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  long long grid = sms < kGridMax ? sms : kGridMax;
+  if (grid > s.units) grid = s.units;
+  if (grid < 1) return cudaSuccess;
+  e = cudaFuncSetAttribute(decode_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_mma_kernel<D><<<(unsigned)grid, kMmaThreads, smem, st>>>(
+      mk, mv, (const __nv_bfloat16*)q, seqlens, Hq, Hkv, Lmax, B, p.width, s.ck, s.subs, stages,
+      s.units, p.parts_max, ws_idx, ws_cnt, ws_part, ws_ctr, (__nv_bfloat16*)O,
+      scale * 1.4426950408889634f);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const void* Kc,
                                    const void* Vc, const float* S, const int32_t* seqlens,
@@ -836,10 +1235,15 @@ static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const voi
       idx_out, 1.0f / sqrtf((float)D));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return p.G <= 4 ? launch_stream<T, D, 4>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale, O,
-                                           ws_idx, ws_cnt, ws_ctr, ws_part, st)
-                  : launch_stream<T, D, 8>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale, O,
-                                           ws_idx, ws_cnt, ws_ctr, ws_part, st);
+  if constexpr (sizeof(T) == 2) {
+    return launch_mma<D>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale, O, ws_idx, ws_cnt,
+                         ws_ctr, ws_part, st);
+  } else {
+    return p.G <= 4 ? launch_stream<T, D, 4>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale,
+                                             O, ws_idx, ws_cnt, ws_ctr, ws_part, st)
+                    : launch_stream<T, D, 8>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale,
+                                             O, ws_idx, ws_cnt, ws_ctr, ws_part, st);
+  }
 }
 
 cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
