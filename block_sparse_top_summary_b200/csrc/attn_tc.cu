@@ -3,16 +3,18 @@
 // "Estágio 2", a FlashAttention-style kernel iterating only the active blocks,
 // here written for sm_100a).
 //
-// Work item (one CTA): 256 query rows that share one block selection, i.e.
-// (batch, KV head g, query block i, group of 256/B query heads of g).  They
-// form two M-tiles of 128 rows (B = 64: two heads x 64 rows; B = 128: one head
-// x 128 rows).  The selected blocks are visited in chunks of 128 keys (two
-// blocks at B = 64, one at B = 128; an odd last block is paired with an
-// all-zero out-of-range box whose keys are masked).
+// Work item: 256 query rows that share one block selection, i.e. (batch, KV
+// head g, query block i, group of 256/B query heads of g).  They form two
+// M-tiles of 128 rows (B = 64: two heads x 64 rows; B = 128: one head x 128
+// rows).  The selected blocks are visited in chunks of 128 keys (two blocks at
+// B = 64, one at B = 128; an odd last block is paired with an all-zero
+// out-of-range box whose keys are masked).  One persistent CTA per SM runs a
+// sequence of work items back to back.
 //
 // Roles (576 threads, 18 warps):
-//   warp 0      TMA producer: Q once (8 boxes of 64 x 64 bf16, 128-byte swizzle),
-//               then K and V of every chunk into a 2-stage ring;
+//   warp 0      TMA producer: Q of each work item (8 boxes of 64 x 64 bf16,
+//               128-byte swizzle), then K and V of every chunk into a 2-stage
+//               ring;
 //   warp 1      TMEM owner (512 columns) and MMA issuer (one thread):
 //               S_t = Q_t K^T  (tcgen05.mma kind::f16, M=128 N=128 K=16, A and B
 //               from shared memory), O_t += P_t V (A = P from TMEM, B = V from
@@ -21,8 +23,9 @@
 //               per row (row = TMEM lane, each thread one 64-key half); read S
 //               (tcgen05.ld), mask (only the last chunk holds the diagonal
 //               block), exchange the half-row maxima through shared memory,
-//               online softmax in the log2 domain with lazy rescaling (O in
-//               TMEM is rescaled only when the row max grows by more than 2^8),
+//               online softmax in the log2 domain (P is computed against a
+//               reference max; O in TMEM is rescaled only when the row max
+//               exceeds it by more than 2^64),
 //               write P as bf16 pairs into the first 32 columns of the thread's
 //               own S half (tcgen05.st), and finally normalise O and store it.
 // TMEM columns: S of tile t at 128 t (P of keys 0-63 at 128 t, of keys 64-127
