@@ -191,6 +191,15 @@ __device__ __forceinline__ void mask32(uint32_t (&v)[32], int col0, const int (&
   }
 }
 
+// Eight 32-bit words w[o .. o+7] to global memory in one 32-byte store (p
+// 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[16], int o) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[o]),
+               "r"(w[o + 1]), "r"(w[o + 2]), "r"(w[o + 3]), "r"(w[o + 4]), "r"(w[o + 5]),
+               "r"(w[o + 6]), "r"(w[o + 7])
+               : "memory");
+}
+
 // p = 2^(s * scale - m) for 32 raw scores, packed as 16 bf16 pairs into w;
 // adds the (fp32) p to acc.
 __device__ __forceinline__ void exp_pack32(const uint32_t (&v)[32], uint32_t (&w)[16], uint64_t s2,
@@ -449,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const uint32_t tS = tmem + lane_off + t * 128 + half * 64;
     const uint32_t tO = tmem + lane_off + 256 + t * 128 + half * 64;
     bool ok = true;
+    const bool o_al32 = (reinterpret_cast<uintptr_t>(O) & 31u) == 0;
     int gc = 0, kq = 0;
     int ns_next = ns_of(blockIdx.x);
     for (int w = blockIdx.x; ok && w < W; w += gridDim.x) {
@@ -602,10 +612,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         for (int e = 0; e < 16; ++e)
           wv[e] = cvt_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
         if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+          if (o_al32) {
+            // 32-byte stores: every write fills a whole sector
+            st_global_v8(orow + q * 32, wv, 0);
+            st_global_v8(orow + q * 32 + 16, wv, 8);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+          }
         }
       }
       // O of this tile is read: the next item's first P.V may overwrite it
