@@ -142,6 +142,19 @@ def test_attention_parity(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters):
     np.testing.assert_allclose(to_f64(lse), rlse, rtol=0, atol=1e-4)
 
 
+@pytest.mark.parametrize("B,N", [(64, 64 * 230 + 37), (128, 128 * 120 + 5)])
+def test_attention_many_items_per_cta(ssa, B, N):
+    # More work items (256 query rows each) than SMs: every persistent CTA of
+    # the tensor-core kernel runs several items back to back, so each item's
+    # Q load, first S and first P.V follow the previous item's last S and
+    # epilogue, with selection lengths that change from item to item and a
+    # ragged last query block.  Every row is compared with the oracle.
+    assert ssa.ssa_sparse_attn_uses_tensor_cores(torch.bfloat16, 8, 2, 128, B)
+    out, lse, ref, rlse = _attn_case(ssa, 1, 8, 2, N, 128, B, 4, "bf16", 4, seed=21)
+    _check_out(to_f64(out), ref, "bf16")
+    np.testing.assert_allclose(to_f64(lse), rlse, rtol=0, atol=1e-4)
+
+
 def test_all_blocks_equals_dense_causal(ssa):
     Q, K, V = planted_prefill(1, 8, 2, 64 * 16, 128, 64, 0, seed=5, dtype="bf16")
     out, _, _, cnt, _ = ssa.prefill(Q.to(DEV), K.to(DEV), V.to(DEV), 64, 1 << 30)
