@@ -101,9 +101,10 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 // are kept, equal scores going to the lower index; the chosen block indices
 // are written to out[0 ..) in ascending order and their number returned.
 // hist: 256 words of shared memory private to this warp.
-// The k-th largest key is found by a 4-pass MSB-first radix select (8 bits
-// per pass); the compaction pass then walks the candidates in index order and
-// takes every key above the threshold plus the first `need` keys equal to it.
+// The k-th largest key is found by an MSB-first radix select, 8 bits per pass,
+// stopping early once the threshold bin holds exactly the keys still needed;
+// the compaction pass then walks the candidates in index order and takes every
+// key above the threshold prefix plus the first `need` keys equal to it.
 __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, int first,
                                                 int32_t* out, uint32_t* hist) {
   const int lane = threadIdx.x & 31;
@@ -150,7 +151,7 @@ __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, i
     const bool mine = (excl < (uint32_t)need) && ((uint32_t)need <= incl);
     const uint32_t who = __ballot_sync(0xffffffffu, mine);
     const int src = __ffs(who) - 1;
-    uint32_t dd = 0, above = 0;
+    uint32_t dd = 0, above = 0, in_bin = 0;
     if (lane == src) {
       uint32_t run = excl;
 #pragma unroll
@@ -158,6 +159,7 @@ __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, i
         if (run + c[q] >= (uint32_t)need) {
           dd = 255u - (uint32_t)(lane * 8 + q);
           above = run;
+          in_bin = c[q];
           break;
         }
         run += c[q];
@@ -165,18 +167,22 @@ __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, i
     }
     dd = __shfl_sync(0xffffffffu, dd, src);
     above = __shfl_sync(0xffffffffu, above, src);
+    in_bin = __shfl_sync(0xffffffffu, in_bin, src);
     prefix |= dd << shift;
     pmask |= 255u << shift;
     need -= (int)above;
     __syncwarp();
+    // every key with this prefix is taken: no tie below it can matter
+    if (in_bin == (uint32_t)need) break;
   }
-  // prefix is now the k-th largest key; take all keys > prefix and the first
-  // `need` keys == prefix in ascending index order.
+  // Take every key whose masked value is above prefix, and the first `need`
+  // keys equal to it in ascending index order (all of them when the passes
+  // stopped early).
   int pos = 0, eq_seen = 0;
   for (int base = 0; base < n; base += 32) {
     const int e = base + lane;
     const bool ok = e < n;
-    const uint32_t key = ok ? order_key(sc[e]) : 0u;
+    const uint32_t key = ok ? (order_key(sc[e]) & pmask) : 0u;
     const bool gt = ok && key > prefix;
     const bool eq = ok && key == prefix;
     const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
