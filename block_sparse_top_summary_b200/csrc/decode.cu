@@ -484,8 +484,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
     const int bg = n < nunits ? (int)((u0 + n) / Ubg) : -2;
     if (bg != cur) {
       if (cur >= 0) {
-        // ---- end of a (sequence, KV head): merge the warps' states.  Round
-        // 1: warps kMW.. publish, warp w < kMW folds in warp w + kMW; round 2:
+        // ---- end of a (sequence, KV head): merge the warps' states.  First
+        // warps kMW.. publish and warp w < kMW folds in warp w + kMW; then
         // warps < kMW publish and every thread merges the kMW slots.
         float l = l_run;
 #pragma unroll
