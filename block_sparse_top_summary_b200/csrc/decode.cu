@@ -504,6 +504,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
                   o2[h][e];
         };
         if (warp >= kMW) publish();
+        __syncwarp();
         consumer_sync();
         if (warp < kMW) {
           float m_new = m_run, l_new = l;
@@ -533,6 +534,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
           __syncwarp();
           publish();
         }
+        __syncwarp();
         consumer_sync();
         const int b = cur / Hkv, g = cur - b * Hkv;
         const long long uf = (long long)cur * Ubg;
@@ -923,6 +925,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
         for (int nt = 0; nt < ON; ++nt)
           *reinterpret_cast<float2*>(ow + ((size_t)warp * 8 + gr) * D + nt * 8 + 2 * tq) =
               make_float2(oc[nt][0], oc[nt][1]);
+        __syncwarp();
         mma_consumer_sync();
         const int b = cur / Hkv, g = cur - b * Hkv;
         const long long uf = (long long)cur * Ubg;
@@ -1062,6 +1065,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
           }
           m_run = cm;
         }
+        __syncwarp();  // reconverge before the warp-collective mma.sync below
         uint32_t pa[NT / 2][2];
 #pragma unroll
         for (int p = 0; p < NT / 2; ++p) {
