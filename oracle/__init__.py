@@ -7,6 +7,7 @@ from .ssa_oracle import (  # noqa: F401
     attention_probs,
     block_summary,
     decode,
+    decode_append,
     decode_route,
     pool_query_blocks,
     route,

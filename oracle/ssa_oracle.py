@@ -25,7 +25,11 @@ What it computes, in the order the pages give the pipeline (DashAttention page,
   page, "Estágio 2");
 * decode: the same stages for one query token at the end of a KV cache
   (DashAttention page, "Contribuições Principais" 4; The Sparse Frontier page,
-  RQ2, decode keeps the whole cache and loads selected pages).
+  RQ2, decode keeps the whole cache and loads selected pages);
+* incremental decoding keeps the cache and its summaries current: each new
+  token's key and value are appended, and a block's summary is formed once
+  the block is complete (DashAttention page, "Contribuições Principais" 4 and
+  "Estágio 0").
 
 Every array is float64.  bf16 and fp32 inputs upcast to float64 exactly.
 Where the pages leave a step open, the reading taken is stated at the function.
@@ -46,6 +50,7 @@ __all__ = [
     "attention_probs",
     "decode_route",
     "decode",
+    "decode_append",
 ]
 
 
@@ -285,3 +290,36 @@ def decode(q, Kc, Vc, seqlens, B: int, topk: int, scale: float | None = None,
             O[bi, g * G : (g + 1) * G] = (e / den) @ Vb[g][kpos]
             LSE[bi, g * G : (g + 1) * G] = (m + np.log(den))[:, 0]
     return O, LSE, idx, cnt
+
+
+def decode_append(Kc, Vc, S, seqlens, k_new, v_new, B: int):
+    """Append one token per sequence to a KV cache and keep its summaries current.
+
+    ``Kc``, ``Vc``: ``[b, Hkv, Lmax, d]``; ``S``: ``[b, Hkv, Lmax // B, d]``;
+    ``seqlens``: ``[b]`` tokens held; ``k_new``, ``v_new``: ``[b, Hkv, d]``.
+    For a sequence holding L tokens, 0 <= L < Lmax, the new row goes to
+    position L and the sequence then holds L + 1 tokens; when L + 1 is a
+    multiple of B, block (L + 1) / B - 1 has just become complete and its
+    summary is the mean of its B keys (the stage-0 summary, formed once a
+    block is complete: DashAttention page, "Estágio 0" and "Contribuições
+    Principais" 4).  A sequence with L outside [0, Lmax) is left unchanged.
+    Returns new ``(Kc, Vc, S, seqlens)`` (float64 copies, seqlens int64).
+    """
+    Kc = _f64(Kc).copy()
+    Vc = _f64(Vc).copy()
+    S = _f64(S).copy()
+    seqlens = np.asarray(seqlens, dtype=np.int64).copy()
+    k_new = _f64(k_new)
+    v_new = _f64(v_new)
+    Lmax = Kc.shape[2]
+    for bi in range(Kc.shape[0]):
+        L = int(seqlens[bi])
+        if not 0 <= L < Lmax:
+            continue
+        Kc[bi, :, L] = k_new[bi]
+        Vc[bi, :, L] = v_new[bi]
+        seqlens[bi] = L + 1
+        if (L + 1) % B == 0:
+            j = (L + 1) // B - 1
+            S[bi, :, j] = Kc[bi, :, j * B : (j + 1) * B].mean(axis=1)
+    return Kc, Vc, S, seqlens

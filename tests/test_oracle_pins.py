@@ -339,3 +339,72 @@ def test_decode_scores_equal_mean_over_group_heads_of_dots():
             for j in range(nb):
                 vals = [float(q[bi, h] @ S[bi, g, j]) / math.sqrt(d) for h in range(g * G, (g + 1) * G)]
                 assert abs(sc[bi, g, j] - sum(vals) / G) < 1e-12
+
+
+# ---------------------------------------------------------------- decode: appending tokens
+def test_append_from_empty_rebuilds_the_cache_and_every_summary():
+    # Appending a cache's rows one by one, starting from empty, must give back
+    # that cache and the summary of every complete block: nothing more, in the
+    # same positions.
+    rng = np.random.default_rng(40)
+    b, h, Lmax, d, B = 2, 3, 40, 4, 8
+    K = rng.integers(-9, 9, size=(b, h, Lmax, d)).astype(np.float64)
+    V = rng.integers(-9, 9, size=(b, h, Lmax, d)).astype(np.float64)
+    Kc = np.zeros_like(K)
+    Vc = np.zeros_like(V)
+    S = np.full((b, h, Lmax // B, d), np.nan)
+    L = np.zeros(b, dtype=np.int64)
+    for t in range(Lmax):
+        Kc, Vc, S, L = O.decode_append(Kc, Vc, S, L, K[:, :, t], V[:, :, t], B)
+        assert L.tolist() == [t + 1] * b
+        done = (t + 1) // B
+        assert np.isnan(S[:, :, done:]).all()  # no summary before its block is complete
+    assert np.array_equal(Kc, K) and np.array_equal(Vc, V)
+    # integer rows: the means are exact, so compare with the closed form directly
+    for j in range(Lmax // B):
+        assert np.array_equal(S[:, :, j], K[:, :, j * B:(j + 1) * B].sum(axis=2) / B)
+
+
+def test_append_arithmetic_block_gives_its_midpoint():
+    # Rows a + r*delta for r = 0..B-1 of one block: its mean is a + (B-1)/2 * delta.
+    b, h, B, d = 1, 2, 16, 3
+    a = np.array([1.0, -2.0, 0.5])
+    delta = np.array([0.25, 1.0, -0.5])
+    Lmax = 2 * B
+    Kc = np.zeros((b, h, Lmax, d))
+    Vc = np.zeros_like(Kc)
+    S = np.zeros((b, h, Lmax // B, d))
+    Kc[:, :, B:2 * B - 1] = a + np.arange(B - 1)[:, None] * delta  # rows B .. 2B-2 already there
+    L = np.array([2 * B - 1])
+    knew = np.broadcast_to(a + (B - 1) * delta, (b, h, d))
+    Kc2, Vc2, S2, L2 = O.decode_append(Kc, Vc, S, L, knew, np.ones((b, h, d)), B)
+    assert L2.tolist() == [2 * B]
+    np.testing.assert_allclose(S2[0, :, 1], np.broadcast_to(a + (B - 1) / 2 * delta, (h, d)),
+                               rtol=0, atol=1e-12)
+    assert np.array_equal(S2[:, :, 0], S[:, :, 0])  # the other block's summary is untouched
+    assert np.array_equal(Vc2[0, :, 2 * B - 1], np.ones((h, d)))
+
+
+def test_append_leaves_incomplete_blocks_and_invalid_lengths_alone():
+    rng = np.random.default_rng(41)
+    b, h, Lmax, d, B = 4, 2, 24, 4, 8
+    Kc = rng.standard_normal((b, h, Lmax, d))
+    Vc = rng.standard_normal((b, h, Lmax, d))
+    S = rng.standard_normal((b, h, Lmax // B, d))
+    L = np.array([3, Lmax, -1, Lmax - 1])
+    kn = rng.standard_normal((b, h, d))
+    vn = rng.standard_normal((b, h, d))
+    Kc2, Vc2, S2, L2 = O.decode_append(Kc, Vc, S, L, kn, vn, B)
+    assert L2.tolist() == [4, Lmax, -1, Lmax]
+    # sequence 0: row 3 written, block 0 not complete, its summary unchanged
+    assert np.array_equal(Kc2[0, :, 3], kn[0]) and np.array_equal(Vc2[0, :, 3], vn[0])
+    assert np.array_equal(S2[0], S[0])
+    # sequences 1 and 2: full cache / negative length, nothing changes
+    for bi in (1, 2):
+        assert np.array_equal(Kc2[bi], Kc[bi]) and np.array_equal(Vc2[bi], Vc[bi])
+        assert np.array_equal(S2[bi], S[bi])
+    # sequence 3: the last row completes the last block, equal to block_summary of the result
+    assert np.array_equal(Kc2[3, :, Lmax - 1], kn[3])
+    np.testing.assert_allclose(S2[3, :, -1], O.block_summary(Kc2[3:4], B)[0, :, -1], rtol=0,
+                               atol=1e-12)
+    assert np.array_equal(S2[3, :, :-1], S[3, :, :-1])
