@@ -13,6 +13,7 @@ from .abi import (  # noqa: F401
     route_width,
     ssa_block_summary,
     ssa_decode,
+    ssa_decode_append,
     ssa_decode_noalloc,
     ssa_decode_workspace_size,
     ssa_device_error,

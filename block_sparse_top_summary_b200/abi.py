@@ -239,6 +239,28 @@ def ssa_decode_noalloc(q, Kc, Vc, S, seqlens, B: int, topk: int, scale: float | 
     return O, idx
 
 
+def ssa_decode_append(Kc, Vc, S, seqlens, k_new, v_new, B: int, stream=None):
+    """Append one token per sequence to the cache, in place.
+
+    Writes ``k_new`` / ``v_new`` ``[batch, Hkv, d]`` at each sequence's length,
+    raises ``seqlens`` by one and refreshes the summary ``S`` of a block the
+    append completes.  Sequences whose cache is full are left unchanged.
+    """
+    for t, n in ((Kc, "Kc"), (Vc, "Vc"), (S, "S"), (seqlens, "seqlens"), (k_new, "k_new"),
+                 (v_new, "v_new")):
+        _need(t, n)
+    lib = load_library()
+    fn = lib.ssa_decode_append
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, vp]
+    fn.restype = i
+    batch, Hkv, Lmax, d = Kc.shape
+    _check("ssa_decode_append", fn(
+        _ptr(Kc), _ptr(Vc), _dtype_code(Kc), _ptr(S), _ptr(seqlens), _ptr(k_new), _ptr(v_new),
+        batch, Hkv, Lmax, d, B, _stream(stream)))
+    return Kc, Vc, S, seqlens
+
+
 # ------------------------------------------------------------- test hooks
 def ssa_debug_wait_timeout(limit_us: int, stream=None):
     """Run the bounded-wait self-test (include/ssa_debug.h); read the result with

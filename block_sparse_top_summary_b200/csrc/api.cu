@@ -132,6 +132,22 @@ ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype d
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ssa_status ssa_decode_append(void* Kc, void* Vc, ssa_dtype dtype, float* S, int32_t* seqlens,
+                             const void* k_new, const void* v_new, int batch, int Hkv, int Lmax,
+                             int d, int B, ssa_stream stream) {
+  ssa_status st = check_dims(d, B, dtype);
+  if (st != SSA_OK) return st;
+  if (batch <= 0 || Hkv <= 0 || Lmax <= 0) return SSA_ERR_INVALID_ARG;
+  if (Kc == nullptr || Vc == nullptr || seqlens == nullptr || k_new == nullptr ||
+      v_new == nullptr)
+    return SSA_ERR_INVALID_ARG;
+  if (Lmax / B > 0 && S == nullptr) return SSA_ERR_INVALID_ARG;
+  if (!aligned16(Kc) || !aligned16(Vc) || !aligned16(S) || !aligned16(k_new) || !aligned16(v_new))
+    return SSA_ERR_INVALID_ARG;
+  return from_cuda(ssa::launch_decode_append(Kc, Vc, dtype, S, seqlens, k_new, v_new, batch, Hkv,
+                                             Lmax, d, B, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ssa_status ssa_device_error(int* code) {
   if (code == nullptr) return SSA_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return SSA_ERR_CUDA;

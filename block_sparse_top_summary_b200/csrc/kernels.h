@@ -49,6 +49,10 @@ cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, co
                           int Hkv, int Lmax, int d, int B, float scale, void* O, int32_t* idx_out,
                           void* ws, cudaStream_t st);
 
+cudaError_t launch_decode_append(void* Kc, void* Vc, ssa_dtype dt, float* S, int32_t* seqlens,
+                                 const void* k_new, const void* v_new, int batch, int Hkv,
+                                 int Lmax, int d, int B, cudaStream_t st);
+
 // Device error words (one per translation unit that has bounded waits):
 // read and reset; returns the first non-zero code or 0.
 int read_and_reset_attn_tc_error();

@@ -163,6 +163,34 @@ ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype d
                       size_t ws_bytes, ssa_stream stream);
 
 /*
+ * Append one token per sequence to the decode KV cache and keep its block
+ * summaries current (DashAttention page, "Contribuições Principais" 4,
+ * incremental decoding; "Estágio 0": a block's summary is the mean of its B
+ * keys, formed once the block is complete).
+ *
+ * For sequence b holding L = seqlens[b] tokens with 0 <= L < Lmax:
+ *   Kc[b, g, L, :] = k_new[b, g, :],  Vc[b, g, L, :] = v_new[b, g, :]  (all g)
+ *   if (L + 1) % B == 0:  S[b, g, (L+1)/B - 1, :] = mean over that block's B
+ *                         keys (fp32 sum, then / B)
+ *   seqlens[b] = L + 1.
+ * A sequence with L outside [0, Lmax) is left unchanged (its cache is full or
+ * its length invalid).  After the call, ssa_decode with the same seqlens
+ * attends the new token as the current one.
+ *
+ * Kc, Vc: [batch, Hkv, Lmax, d] of `dtype` (modified in place);
+ * S: [batch, Hkv, Lmax / B, d] fp32 (modified in place; may be NULL only if
+ *    Lmax < B);
+ * seqlens: [batch] int32 (read and raised in place, on the device);
+ * k_new, v_new: [batch, Hkv, d] of `dtype`.
+ * All device pointers, 16-byte aligned.  Supported: d in {64, 128}; B a
+ * multiple of 16 in [16, 128].  Calls on one cache must not overlap on the
+ * device.
+ */
+ssa_status ssa_decode_append(void* Kc, void* Vc, ssa_dtype dtype, float* S, int32_t* seqlens,
+                             const void* k_new, const void* v_new, int batch, int Hkv, int Lmax,
+                             int d, int B, ssa_stream stream);
+
+/*
  * Largest scratch area ssa_decode_noalloc can use (40 MiB).
  */
 #define SSA_DECODE_NOALLOC_MAX_BYTES ((size_t)40 << 20)

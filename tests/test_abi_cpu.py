@@ -103,6 +103,31 @@ def test_decode_workspace_and_rejections(lib):
     assert r == 1  # workspace not 256-byte aligned
 
 
+def test_decode_append_rejections(lib):
+    fn = lib.ssa_decode_append
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, vp]
+    fn.restype = i
+    ok = (FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 4, 2, 1024, 128, 64, NULL)
+
+    def call(**kw):
+        args = list(ok)
+        for k, v in kw.items():
+            args[{"Kc": 0, "Vc": 1, "dt": 2, "S": 3, "L": 4, "kn": 5, "vn": 6, "batch": 7,
+                  "Hkv": 8, "Lmax": 9, "d": 10, "B": 11}[k]] = v
+        return fn(*args)
+
+    assert call(d=96) == 2                   # d not 64 or 128
+    assert call(B=40) == 2                   # B not a multiple of 16
+    assert call(dt=7) == 1                   # unknown dtype
+    assert call(batch=0) == 1
+    assert call(Lmax=0) == 1
+    assert call(Kc=NULL) == 1
+    assert call(L=NULL) == 1
+    assert call(S=NULL) == 1                 # the cache holds complete blocks
+    assert call(kn=ctypes.c_void_p(0x100008)) == 1  # not 16-byte aligned
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(ImportError):
         abi.load_library(str(tmp_path / "missing.so"))

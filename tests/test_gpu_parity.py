@@ -282,3 +282,58 @@ def test_large_score_jump_in_a_later_block(ssa, B):
     ref, rlse = O.sparse_attention(to_f64(Q), to_f64(K), to_f64(V), gi, cnt.cpu().numpy(), B)
     _check_out(to_f64(out), ref, "bf16")
     assert np.max(np.abs(to_f64(lse) - rlse)) < 1e-2
+
+
+# ---------------------------------------------------------------- decode: appending tokens
+@pytest.mark.parametrize("dtype,d,B", [("bf16", 128, 64), ("f32", 64, 16), ("bf16", 64, 128),
+                                       ("f32", 128, 32)])
+def test_decode_append_parity(ssa, dtype, d, B):
+    # lengths: completing a block, mid-block, empty, full cache, last free slot
+    batch, Hkv, Lmax = 5, 3, B * 6
+    gen = torch.Generator().manual_seed(31)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    Kc = torch.randn(batch, Hkv, Lmax, d, generator=gen).to(tdt)
+    Vc = torch.randn(batch, Hkv, Lmax, d, generator=gen).to(tdt)
+    S = torch.randn(batch, Hkv, Lmax // B, d, generator=gen)
+    L = torch.tensor([2 * B - 1, 3 * B + 5, 0, Lmax, Lmax - 1], dtype=torch.int32)
+    kn = torch.randn(batch, Hkv, d, generator=gen).to(tdt)
+    vn = torch.randn(batch, Hkv, d, generator=gen).to(tdt)
+    rK, rV, rS, rL = O.decode_append(to_f64(Kc), to_f64(Vc), S.double().numpy(), L.numpy(),
+                                     to_f64(kn), to_f64(vn), B)
+    Kd, Vd, Sd, Ld = Kc.to(DEV), Vc.to(DEV), S.to(DEV), L.to(DEV)
+    ssa.ssa_decode_append(Kd, Vd, Sd, Ld, kn.to(DEV), vn.to(DEV), B)
+    assert Ld.cpu().tolist() == rL.tolist()
+    assert np.array_equal(to_f64(Kd.cpu()), rK) and np.array_equal(to_f64(Vd.cpu()), rV)
+    got = Sd.cpu().double().numpy()
+    np.testing.assert_allclose(got, rS, rtol=0, atol=F32_MAX_ABS)
+    changed = np.abs(rS - S.double().numpy()).max(axis=-1) > 0
+    assert np.array_equal(got[~changed], S.double().numpy()[~changed])  # the rest untouched, bitwise
+
+
+def test_append_then_decode_matches_oracle(ssa):
+    # A serving loop: three appends, one of which completes a block, then one
+    # decode step on the grown caches.
+    B, topk = 64, 3
+    q, Kc, Vc, L = planted_decode(2, 8, 2, B * 20, 128, B, 3, seed=12, dtype="bf16",
+                                  seqlens=[B * 5 - 2, B * 11 + 7])
+    Kd, Vd, Ld = Kc.to(DEV), Vc.to(DEV), L.to(DEV)
+    Sd = ssa.ssa_block_summary(Kd, B)
+    rK, rV, rS, rL = to_f64(Kc), to_f64(Vc), Sd.cpu().double().numpy(), L.numpy()
+    gen = torch.Generator().manual_seed(13)
+    for _ in range(3):
+        kn = torch.randn(2, 2, 128, generator=gen).to(torch.bfloat16)
+        vn = torch.randn(2, 2, 128, generator=gen).to(torch.bfloat16)
+        ssa.ssa_decode_append(Kd, Vd, Sd, Ld, kn.to(DEV), vn.to(DEV), B)
+        rK, rV, rS, rL = O.decode_append(rK, rV, rS, rL, to_f64(kn), to_f64(vn), B)
+    assert Ld.cpu().tolist() == rL.tolist() == [B * 5 + 1, B * 11 + 10]
+    np.testing.assert_allclose(Sd.cpu().double().numpy()[0, :, 4], O.block_summary(rK[:1], B)[0, :, 4],
+                               rtol=0, atol=F32_MAX_ABS)  # the block the second append completed
+    out, idx = ssa.ssa_decode(q.to(DEV), Kd, Vd, Sd, Ld, B, topk)
+    gi = idx.cpu().numpy()
+    gc = (gi >= 0).sum(-1)
+    oi, oc, osc = O.decode_route(to_f64(q), rS, rL, B, topk)
+    rows, near, bad = compare_selection(gi, gc, oi, oc,
+                                        lambda r: {j: osc[r][j] for j in range(osc.shape[-1])})
+    assert not bad, bad[:3]
+    ref, _, _, _ = O.decode(to_f64(q), rK, rV, rL, B, topk, idx=gi, cnt=gc)
+    _check_out(to_f64(out), ref, "bf16")
