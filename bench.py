@@ -311,6 +311,40 @@ def run_ours(args, world, rank, local):
     h2d = (Q.numel() + K.numel() + V.numel() + q.numel()) * 2 + L.numel() * 4
     d2h = Q.numel() * 2 + q.numel() * 2
 
+    # --- appending one token per sequence (incremental decoding), timed on its
+    # own after everything else, as it rewrites a cache row.  Every call is
+    # set up so that its append completes a block (the costlier case): 20
+    # calls, each with its own copy of the lengths, are captured in a CUDA graph
+    # and replayed, so the device time carries no host gaps; the lengths are
+    # restored between replays, outside the timed events.
+    app_len = torch.full_like(L, (cd.L // cd.B - 1) * cd.B - 1)
+    app_Ls = [app_len.clone() for _ in range(20)]
+    kn = torch.randn(cd.batch, cd.Hkv, cd.d, device=q.device).to(torch.bfloat16)
+    vn = torch.randn(cd.batch, cd.Hkv, cd.d, device=q.device).to(torch.bfloat16)
+    ssa.ssa_decode_append(Kc, Vc, Sc, app_Ls[0], kn, vn, cd.B, stream=stream)  # warm-up
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for t_ in app_Ls:
+            ssa.ssa_decode_append(Kc, Vc, Sc, t_, kn, vn, cd.B)
+    app_ms = []
+    for it in range(3 + 10):
+        for t_ in app_Ls:
+            t_.copy_(app_len)
+        torch.cuda.synchronize()
+        a, b_ = ev(), ev()
+        a.record(stream)
+        graph.replay()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        if it >= 3:
+            app_ms.append(a.elapsed_time(b_) / len(app_Ls))
+    del graph
+    app_ms = max_over_ranks(float(np.mean(app_ms)), world)
+    # per sequence and KV head: two rows written, the completed block's B key rows
+    # read back, one fp32 summary row written
+    app_bytes = cd.batch * cd.Hkv * (2 * cd.d * 2 + cd.B * cd.d * 2 + cd.d * 4)
+
     tc = ssa.ssa_sparse_attn_uses_tensor_cores(Q.dtype, cp.Hq, cp.Hkv, cp.d, cp.B)
     kernels = {
         "ssa_block_summary": {"ms": float(seg_mean[0]), "bound": "hbm",
@@ -321,6 +355,10 @@ def run_ours(args, world, rank, local):
                                 "TFLOP/s": attn_tflops},
         "ssa_decode": {"ms": float(seg_mean[3]), "bound": "hbm", "GB/s": dec_gbs,
                        "tokens/s": dec_tok},
+        "ssa_decode_append": {"ms": app_ms, "bound": "hbm",
+                              "GB/s": app_bytes / (app_ms * 1e-3) / 1e9,
+                              "note": "timed apart from the step (CUDA graph of 20 calls); "
+                                      "every append completes a block"},
     }
     for k, v in kernels.items():
         if "GB/s" in v:
