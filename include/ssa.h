@@ -17,7 +17,8 @@
  *   (grouped-query attention, GQA).
  * - Every pointer argument is a DEVICE pointer, 16-byte aligned, owned by the
  *   caller.  The library allocates and frees nothing and keeps no state between
- *   calls other than a device-side error word (see ssa_device_error).
+ *   calls other than a device-side error word (see ssa_device_error) and the
+ *   fixed scratch array of ssa_decode_noalloc.
  * - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *   stream) and nothing synchronises with the host.
  * - Argument checks run on the host before any launch; a failed check returns
