@@ -311,6 +311,31 @@ __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity
   return ok != 0;
 }
 
+// Warp-uniform bounded wait until the shared word `tag` equals `want`
+// (acquire order); false when the CTA aborted or the wait expired.
+__device__ __forceinline__ bool warp_wait_tag(const int* tag, int want, volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0 && ptx::ld_acquire_s32(tag) != want) {
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (ptx::ld_acquire_s32(tag) == want) break;
+      if ((it & 255u) == 0) {
+        if (*abort) {
+          ok = 0;
+          break;
+        }
+        if (globaltimer_ns() - t0 > kWaitNs) {
+          *abort = 1;
+          atomicCAS(&g_decode_error, 0, (int)SSA_ERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -808,6 +833,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ int info[kMaxStages];
+  __shared__ int tag[kMaxStages];  // unit each stage was last refilled for
   __shared__ int s_abort, s_last;
 
   const int G = Hq / Hkv;
@@ -828,6 +854,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
+      tag[s] = -1;
     }
     s_abort = 0;
     ptx::fence_mbar_init();
@@ -873,6 +900,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
           break;
         if (lane == 0) {
           info[st] = rows;
+          ptx::st_release_s32(&tag[st], n);
           if (rows > 0) {
             const int bg = (int)((u0 + n) / Ubg);
             unsigned char* dst = base + (size_t)st * stage_bytes;
@@ -1005,8 +1033,14 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
     if (n % kMmaCW != warp) continue;
 
     // ---- one unit
+    // Stage st holds units n - stages, n, n + stages ... and the unit before
+    // this one there belongs to another warp when kMmaCW does not divide
+    // stages.  A parity wait cannot tell that unit's phase, still open, from
+    // this unit's, complete; the producer tags the stage with n only after
+    // that unit was consumed, so wait for the tag first.
     const int st = n % stages;
-    if (warp_wait_bounded(&full[st], (uint32_t)(n / stages) & 1u, abort)) {
+    if (warp_wait_tag(&tag[st], n, abort) &&
+        warp_wait_bounded(&full[st], (uint32_t)(n / stages) & 1u, abort)) {
       const int rows = info[st];
       if (rows > 0) {
         unsigned char* stg = base + (size_t)st * stage_bytes;
