@@ -13,5 +13,6 @@ from .ssa_oracle import (  # noqa: F401
     route,
     select_topk,
     sparse_attention,
+    sparse_attention_backward,
     summary_scores,
 )

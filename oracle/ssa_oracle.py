@@ -29,7 +29,13 @@ What it computes, in the order the pages give the pipeline (DashAttention page,
 * incremental decoding keeps the cache and its summaries current: each new
   token's key and value are appended, and a block's summary is formed once
   the block is complete (DashAttention page, "Contribuições Principais" 4 and
-  "Estágio 0").
+  "Estágio 0");
+* training: the backward pass of stage 2.  The hard top-k selection passes
+  no gradient to the routing or the summaries (DashAttention page,
+  "Declaração do Problema" 2), and keys outside the selected blocks get zero
+  gradient (SSA page, "1. Definição do Problema" 2; AdaSplash-2 page,
+  "4. Resultados Experimentais": the backward skips zero-gradient blocks).
+  So the gradients are those of stage 2 with the selection held fixed.
 
 Every array is float64.  bf16 and fp32 inputs upcast to float64 exactly.
 Where the pages leave a step open, the reading taken is stated at the function.
@@ -51,6 +57,7 @@ __all__ = [
     "decode_route",
     "decode",
     "decode_append",
+    "sparse_attention_backward",
 ]
 
 
@@ -192,6 +199,60 @@ def sparse_attention(Q, K, V, idx, cnt, B: int, scale: float | None = None,
         O[bi, g * G : (g + 1) * G, t0:t1, :] = np.einsum("hrk,kd->hrd", p, V[bi, g][kpos])
         LSE[bi, g * G : (g + 1) * G, t0:t1] = (m + np.log(den))[..., 0]
     return O, LSE
+
+
+def sparse_attention_backward(Q, K, V, idx, cnt, dO, B: int, scale: float | None = None):
+    """Gradients of :func:`sparse_attention`'s ``O`` with the selection fixed.
+
+    Given the upstream gradient ``dO`` ``[b, Hq, N, d]``, returns
+    ``(dQ, dK, dV)`` with the shapes of Q, K and V.  Per unit (b, g, i), P is
+    the unit's softmax over its selected, causally visible keys, and with
+    ``O = P V``:
+
+    * ``dV[keys] += P^T dO``;
+    * ``dS = P * (dO V^T - rowsum(dO * O))``, the softmax Jacobian applied to
+      ``dP = dO V^T``;
+    * ``dQ = scale * dS K[keys]`` and ``dK[keys] += scale * dS^T Q``.
+
+    dK and dV sum over the G query heads that share the KV head and over the
+    query blocks that selected the key.  Keys that no unit selected, and
+    positions after every query that sees them, get exactly 0.
+    """
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    dO = _f64(dO)
+    b, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    nq = -(-N // B)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    for bi in range(b):
+        for g in range(Hkv):
+            for i in range(nq):
+                sel = [int(j) for j in idx[bi, g, i, : cnt[bi, g, i]]]
+                kpos = _selected_keys(sel, B, N)
+                t0, t1 = i * B, min(N, (i + 1) * B)
+                qpos = np.arange(t0, t1)
+                q = Q[bi, g * G : (g + 1) * G, t0:t1, :]    # [G, r, d]
+                do = dO[bi, g * G : (g + 1) * G, t0:t1, :]  # [G, r, d]
+                k = K[bi, g][kpos]                          # [n, d]
+                v = V[bi, g][kpos]
+                logits = np.einsum("hrd,kd->hrk", q, k) * scale
+                logits = np.where(kpos[None, None, :] > qpos[None, :, None], -np.inf, logits)
+                e = np.exp(logits - logits.max(axis=-1, keepdims=True))
+                p = e / e.sum(axis=-1, keepdims=True)       # [G, r, n]
+                o = np.einsum("hrk,kd->hrd", p, v)
+                dp = np.einsum("hrd,kd->hrk", do, v)
+                ds = p * (dp - np.einsum("hrd,hrd->hr", do, o)[..., None])
+                dQ[bi, g * G : (g + 1) * G, t0:t1, :] = scale * np.einsum("hrk,kd->hrd", ds, k)
+                dK[bi, g, kpos] += scale * np.einsum("hrk,hrd->kd", ds, q)
+                dV[bi, g, kpos] += np.einsum("hrk,hrd->kd", p, do)
+    return dQ, dK, dV
 
 
 def attention_probs(Q, K, idx, cnt, B: int, scale: float | None = None) -> np.ndarray:

@@ -268,6 +268,100 @@ def test_error_bound_linear_in_dropped_mass():
             assert err <= 2 * delta * vmax + 1e-12
 
 
+# ------------------------------------------------- stage 2: backward pass
+@pytest.mark.parametrize("N,B", [(128, 32), (16 * 5 + 7, 16)])
+def test_backward_all_blocks_equals_autograd_of_dense_causal_sdpa(N, B):
+    rng = np.random.default_rng(11)
+    b, Hq, Hkv, d = 2, 4, 2, 16
+    Q, K, V = (rng.standard_normal((b, h, N, d)) for h in (Hq, Hkv, Hkv))
+    dO = rng.standard_normal((b, Hq, N, d))
+    S = O.block_summary(K, B)
+    idx, cnt, _ = O.route(Q, S, B, 10**6, Hkv)
+    dQ, dK, dV = O.sparse_attention_backward(Q, K, V, idx, cnt, dO, B)
+    q, k, v = (torch.from_numpy(x).requires_grad_() for x in (Q, K, V))
+    G = Hq // Hkv
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q, k.repeat_interleave(G, 1), v.repeat_interleave(G, 1), is_causal=True)
+    (out * torch.from_numpy(dO)).sum().backward()
+    for mine, ref in ((dQ, q.grad), (dK, k.grad), (dV, v.grad)):
+        ref = ref.numpy()
+        assert np.max(np.abs(mine - ref)) / np.max(np.abs(ref)) < 1e-12
+
+
+def _loss(Q, K, V, idx, cnt, dO, B):
+    out, _ = O.sparse_attention(Q, K, V, idx, cnt, B)
+    return float(np.sum(out * dO))
+
+
+def test_backward_matches_central_differences_with_fixed_selection():
+    Q, K, V, idx, cnt, B = _tiny_case(seed=12, k=2)
+    rng = np.random.default_rng(13)
+    dO = rng.standard_normal(Q.shape)
+    grads = O.sparse_attention_backward(Q, K, V, idx, cnt, dO, B)
+    eps = 1e-5
+    for which in range(3):
+        for _ in range(3):
+            u = rng.standard_normal(grads[which].shape)
+            xs_p = [Q, K, V]
+            xs_m = [Q, K, V]
+            xs_p[which] = xs_p[which] + eps * u
+            xs_m[which] = xs_m[which] - eps * u
+            fd = (_loss(*xs_p, idx, cnt, dO, B) - _loss(*xs_m, idx, cnt, dO, B)) / (2 * eps)
+            an = float(np.sum(grads[which] * u))
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(an))
+
+
+def test_backward_gradient_stays_inside_one_blocks_selection():
+    # dO nonzero on query block i only: dQ lives on block i's rows, dK and dV
+    # on the keys block i attends (its selected blocks, the diagonal block up
+    # to its last row) and are exactly 0 elsewhere.
+    Q, K, V, idx, cnt, B = _tiny_case(seed=14, k=2)
+    rng = np.random.default_rng(15)
+    N = Q.shape[2]
+    G = Q.shape[1] // K.shape[1]
+    for i in (3, 6, (N - 1) // B):
+        dO = np.zeros(Q.shape)
+        t0, t1 = i * B, min(N, (i + 1) * B)
+        dO[:, :, t0:t1] = rng.standard_normal((Q.shape[0], Q.shape[1], t1 - t0, Q.shape[3]))
+        dQ, dK, dV = O.sparse_attention_backward(Q, K, V, idx, cnt, dO, B)
+        rows = np.zeros(N, bool)
+        rows[t0:t1] = True
+        assert np.all(dQ[:, :, ~rows] == 0.0) and np.any(dQ[:, :, rows] != 0.0)
+        for g in range(K.shape[1]):
+            seen = np.zeros(N, bool)
+            for j in idx[0, g, i, : cnt[0, g, i]]:
+                seen[j * B : min(N, (j + 1) * B)] = True
+            seen[t1:] = False
+            assert np.all(dK[0, g, ~seen] == 0.0) and np.all(dV[0, g, ~seen] == 0.0)
+            assert np.all(np.any(dV[0, g, seen] != 0.0, axis=-1))
+        assert G > 1
+
+
+def test_backward_key_and_value_gradient_sums():
+    # Each softmax row sums to 1, so its Jacobian rows sum to 0: summed over
+    # every key, dK vanishes and dV equals the sum of dO over the group.
+    Q, K, V, idx, cnt, B = _tiny_case(seed=16, k=3)
+    dO = np.random.default_rng(17).standard_normal(Q.shape)
+    _, dK, dV = O.sparse_attention_backward(Q, K, V, idx, cnt, dO, B)
+    G = Q.shape[1] // K.shape[1]
+    for g in range(K.shape[1]):
+        np.testing.assert_allclose(dK[0, g].sum(0), 0.0, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dV[0, g].sum(0), dO[0, g * G : (g + 1) * G].sum((0, 1)),
+                                   rtol=0, atol=1e-11)
+
+
+def test_backward_value_shift_leaves_gradients_unchanged():
+    # V + c shifts every output row by c and dO . O by dO . c, which cancels
+    # in dS, so dQ and dK stay; dV = P^T dO does not read V.
+    Q, K, V, idx, cnt, B = _tiny_case(seed=18, k=2)
+    dO = np.random.default_rng(19).standard_normal(Q.shape)
+    c = np.random.default_rng(20).standard_normal(V.shape[-1]) * 5.0
+    a = O.sparse_attention_backward(Q, K, V, idx, cnt, dO, B)
+    s = O.sparse_attention_backward(Q, K, V + c, idx, cnt, dO, B)
+    for x, y in zip(a, s):
+        np.testing.assert_allclose(x, y, rtol=0, atol=1e-11)
+
+
 # ------------------------------------------------------------------ decode
 def test_decode_all_blocks_equals_dense_last_row():
     q, Kc, Vc, L = planted_decode(3, 4, 2, 200, 16, 16, clusters=3, seed=9, dtype="f32",
