@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(
         const int kk = c / CPR;
         const int cc = c - kk * CPR;
         float fk[EPC], fv[EPC];
-        if (kb + kk < N) {
+        if (kb + kk < N && kc + kk < B) {
           unpack16(ldg16(K + (kvbase + kb + kk) * D + cc * EPC), fk, (const T*)nullptr);
           unpack16(ldg16(V + (kvbase + kb + kk) * D + cc * EPC), fv, (const T*)nullptr);
         } else {
@@ -101,8 +101,10 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(
           a = fmaf(q[e + 3], kv.w, a);
         }
         if (TPR == 2) a += __shfl_xor_sync(0xffffffffu, a, 1);
+        // a chunk may reach past block j (B not a multiple of KC): those keys
+        // belong to the next block, which this row did not select
         const int kpos = kb + kk;
-        sc[kk] = (kpos <= qpos) ? a : -INFINITY;
+        sc[kk] = (kpos <= qpos && kc + kk < B) ? a : -INFINITY;
         cmax = fmaxf(cmax, sc[kk]);
       }
       const float mnew = fmaxf(m, cmax);

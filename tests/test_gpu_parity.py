@@ -135,6 +135,8 @@ def _attn_case(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters, seed=3):
     (1, 8, 2, 128 * 9, 128, 128, 3, "bf16", 3),       # bf16, B = 128
     (1, 4, 4, 32 * 20 + 31, 64, 32, 5, "bf16", 3),    # G = 1, B = 32, d = 64
     (1, 8, 1, 64 * 10, 128, 64, 1 << 30, "bf16", 0),  # all blocks (dense), G = 8
+    (1, 4, 2, 16 * 40 + 5, 64, 16, 4, "bf16", 3),     # B = 16: half a key chunk
+    (1, 2, 1, 48 * 12 + 7, 128, 48, 3, "f32", 2),     # B = 48: chunks straddle blocks
 ])
 def test_attention_parity(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters):
     out, lse, ref, rlse = _attn_case(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters)
