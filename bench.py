@@ -34,7 +34,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import CONFIGS, planted_decode, planted_prefill  # noqa: E402
+from workloads import CONFIGS, planted_decode, planted_prefill, upstream_grad  # noqa: E402
 
 METRIC = "prefill selected-block TFLOP/s & % BF16 peak; decode tokens/s & HBM GB/s"
 
@@ -345,6 +345,31 @@ def run_ours(args, world, rank, local):
     # read back, one fp32 summary row written
     app_bytes = cd.batch * cd.Hkv * (2 * cd.d * 2 + cd.B * cd.d * 2 + cd.d * 4)
 
+    # --- backward of the attention (training), timed apart from the step on the
+    # step's own selection, O and log-sum-exp
+    dOd = upstream_grad(cp.batch, cp.Hq, cp.N, cp.d, seed=rank_seed(cp.seed + 1, rank),
+                        dtype=cp.dtype, device=dev)
+    dQb, dKb, dVb = torch.empty_like(Qd), torch.empty_like(Kd), torch.empty_like(Vd)
+    delta = torch.empty(cp.batch, cp.Hq, cp.N, dtype=torch.float32, device=dev)
+
+    def bwd():
+        ssa.ssa_sparse_attn_bwd(Qd, Kd, Vd, Od, dOd, lse, idx, cnt, cp.B, dQ=dQb, dK=dKb, dV=dVb,
+                                delta=delta)
+
+    bwd_ms = []
+    for it in range(2 + 5):
+        a, b_ = ev(), ev()
+        a.record(stream)
+        bwd()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        if it >= 2:
+            bwd_ms.append(a.elapsed_time(b_))
+    bwd_ms = max_over_ranks(float(np.mean(bwd_ms)), world)
+    # 8 d per unmasked (query, key) pair: the dV, dP, dQ and dK contractions
+    bwd_flops = 2.0 * flops
+    bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
+
     tc = ssa.ssa_sparse_attn_uses_tensor_cores(Q.dtype, cp.Hq, cp.Hkv, cp.d, cp.B)
     kernels = {
         "ssa_block_summary": {"ms": float(seg_mean[0]), "bound": "hbm",
@@ -359,6 +384,11 @@ def run_ours(args, world, rank, local):
                               "GB/s": app_bytes / (app_ms * 1e-3) / 1e9,
                               "note": "timed apart from the step (CUDA graph of 20 calls); "
                                       "every append completes a block"},
+        "ssa_sparse_attn_bwd": {"ms": bwd_ms, "bound": "tensor", "TFLOP/s": bwd_tflops,
+                                "frac_bf16": bwd_tflops / bf16_peak,
+                                "work_per_launch": f"{bwd_flops:.4e} FLOP",
+                                "note": "timed apart from the step; FLOPs = 8 d per unmasked "
+                                        "(query, key) pair, the recomputed S not counted"},
     }
     for k, v in kernels.items():
         if "GB/s" in v:

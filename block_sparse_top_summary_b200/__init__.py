@@ -18,6 +18,7 @@ from .abi import (  # noqa: F401
     ssa_decode_workspace_size,
     ssa_device_error,
     ssa_route,
+    ssa_sparse_attn_bwd,
     ssa_sparse_attn_fwd,
     ssa_sparse_attn_uses_tensor_cores,
 )

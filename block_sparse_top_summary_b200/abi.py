@@ -25,7 +25,7 @@ _STATUS = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED", 3: "
 # Every symbol include/ssa.h declares.
 EXPORTS = ("ssa_status_string", "ssa_version", "ssa_block_summary", "ssa_route",
            "ssa_sparse_attn_fwd", "ssa_sparse_attn_uses_tensor_cores", "ssa_decode_workspace_size",
-           "ssa_decode", "ssa_device_error")
+           "ssa_decode", "ssa_device_error", "ssa_sparse_attn_bwd")
 
 
 class SSAError(RuntimeError):
@@ -259,6 +259,38 @@ def ssa_decode_append(Kc, Vc, S, seqlens, k_new, v_new, B: int, stream=None):
         _ptr(Kc), _ptr(Vc), _dtype_code(Kc), _ptr(S), _ptr(seqlens), _ptr(k_new), _ptr(v_new),
         batch, Hkv, Lmax, d, B, _stream(stream)))
     return Kc, Vc, S, seqlens
+
+
+def ssa_sparse_attn_bwd(Q, K, V, O, dO, lse, idx, cnt, B: int, scale: float | None = None,
+                        dQ=None, dK=None, dV=None, delta=None, stream=None):
+    """Gradients of the selected-block attention: returns ``(dQ, dK, dV)``.
+
+    ``O`` and ``lse`` are the outputs of ``ssa_sparse_attn_fwd`` on the same
+    ``Q, K, V, idx, cnt``; ``dO`` is the gradient of the loss with respect to
+    ``O``.  ``delta`` (``[batch, Hq, N]`` fp32) is scratch.
+    """
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O"), (dO, "dO"), (lse, "lse"), (idx, "idx"),
+                 (cnt, "cnt")):
+        _need(t, n)
+    lib = load_library()
+    fn = lib.ssa_sparse_attn_bwd
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, vp, vp]
+    fn.restype = i
+    batch, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    if delta is None:
+        delta = torch.empty(batch, Hq, N, dtype=torch.float32, device=Q.device)
+    _check("ssa_sparse_attn_bwd", fn(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(lse), _dtype_code(Q), _ptr(idx),
+        _ptr(cnt), batch, Hq, Hkv, N, d, B, idx.shape[-1], ctypes.c_float(scale), _ptr(dQ),
+        _ptr(dK), _ptr(dV), _ptr(delta), _stream(stream)))
+    return dQ, dK, dV
 
 
 # ------------------------------------------------------------- test hooks

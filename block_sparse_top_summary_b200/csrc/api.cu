@@ -91,6 +91,32 @@ ssa_status ssa_sparse_attn_fwd(const void* Q, const void* K, const void* V, ssa_
                                          max_sel, scale, O, lse, s));
 }
 
+ssa_status ssa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O,
+                               const void* dO, const float* lse, ssa_dtype dtype,
+                               const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
+                               int N, int d, int B, int max_sel, float scale, void* dQ, void* dK,
+                               void* dV, float* delta, ssa_stream stream) {
+  ssa_status st = check_dims(d, B, dtype);
+  if (st != SSA_OK) return st;
+  if (dtype != SSA_BF16) return SSA_ERR_UNSUPPORTED;
+  if (batch <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || max_sel < 1) return SSA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) return SSA_ERR_INVALID_ARG;
+  if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr || dO == nullptr ||
+      lse == nullptr || idx == nullptr || cnt == nullptr || dQ == nullptr || dK == nullptr ||
+      dV == nullptr || delta == nullptr)
+    return SSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return SSA_ERR_INVALID_ARG;
+  const long long nq = ((long long)N + B - 1) / B;
+  if ((long long)batch * Hq * nq > 0x7fffffffLL || (long long)batch * Hq * N / 8 > 0x7fffffffLL)
+    return SSA_ERR_UNSUPPORTED;
+  return from_cuda(ssa::launch_attn_bwd(Q, K, V, O, dO, lse, idx, cnt, batch, Hq, Hkv, N, d, B,
+                                        max_sel, scale, dQ, dK, dV, delta,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int ssa_sparse_attn_uses_tensor_cores(ssa_dtype dtype, int Hq, int Hkv, int d, int B) {
   if (!dtype_ok(dtype) || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
   return ssa::attn_tc_supported(dtype, Hq, Hkv, d, B) ? 1 : 0;

@@ -32,6 +32,14 @@ cudaError_t launch_attn_simt(const void* Q, const void* K, const void* V, ssa_dt
                              int N, int d, int B, int max_sel, float scale, void* O, float* lse,
                              cudaStream_t st);
 
+// Backward pass of stage 2 (bf16, mma.sync tiles): delta, dQ, dK, dV.
+size_t attn_bwd_smem_bytes(int d, int B);
+cudaError_t launch_attn_bwd(const void* Q, const void* K, const void* V, const void* O,
+                            const void* dO, const float* lse, const int32_t* idx,
+                            const int32_t* cnt, int batch, int Hq, int Hkv, int N, int d, int B,
+                            int max_sel, float scale, void* dQ, void* dK, void* dV, float* delta,
+                            cudaStream_t st);
+
 // Decode: scratch layout and launch.
 struct DecodePlan {
   int G;          // query heads per KV head

@@ -122,6 +122,37 @@ ssa_status ssa_sparse_attn_fwd(const void* Q, const void* K, const void* V, ssa_
                                ssa_stream stream);
 
 /*
+ * Backward pass of stage 2 with the selection held fixed (DashAttention page,
+ * "Declaração do Problema" 2: hard top-k passes no gradient to the routing;
+ * SSA page, "1. Definição do Problema" 2: keys outside the selected blocks get
+ * zero gradient; AdaSplash-2 page, "4. Resultados Experimentais": the backward
+ * skips the zero blocks).
+ *
+ * With P the softmax of ssa_sparse_attn_fwd (rebuilt as exp(scale q.k - lse))
+ * and dO the gradient of the loss with respect to O:
+ *   delta[b, h, t] = dO[b, h, t, :] . O[b, h, t, :]
+ *   dS             = P * (dO V_sel^T - delta)
+ *   dQ             = scale * dS K_sel
+ *   dK[b, g]      += scale * dS^T Q,   dV[b, g] += P^T dO
+ * dK and dV sum over the query heads of group g and over every query block
+ * whose selection holds the key's block; keys no query sees get 0.  Every
+ * output element is written exactly once, in a fixed summation order (no
+ * atomics), so the result is deterministic.
+ *
+ * Q, O, dO, dQ: [batch, Hq, N, d]; K, V, dK, dV: [batch, Hkv, N, d]; all bf16
+ * (SSA_ERR_UNSUPPORTED for SSA_F32).  lse: [batch, Hq, N] fp32 as written by
+ * ssa_sparse_attn_fwd; idx/cnt: as written by ssa_route (ascending entries).
+ * delta: caller-owned fp32 scratch of batch * Hq * N floats (overwritten).
+ * The contractions run on mma.sync tensor-core tiles (bf16 in, fp32
+ * accumulate); P and dS are rounded to bf16 as operands, outputs to bf16.
+ */
+ssa_status ssa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O,
+                               const void* dO, const float* lse, ssa_dtype dtype,
+                               const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
+                               int N, int d, int B, int max_sel, float scale, void* dQ, void* dK,
+                               void* dV, float* delta, ssa_stream stream);
+
+/*
  * 1 if ssa_sparse_attn_fwd runs this shape on the tensor cores, else 0 (the
  * SIMT kernel).  Pure host query.
  */

@@ -128,6 +128,35 @@ def test_decode_append_rejections(lib):
     assert call(kn=ctypes.c_void_p(0x100008)) == 1  # not 16-byte aligned
 
 
+def test_attention_backward_rejections(lib):
+    fn = lib.ssa_sparse_attn_bwd
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, vp, vp]
+    fn.restype = i
+    names = ["Q", "K", "V", "O", "dO", "lse", "dt", "idx", "cnt", "batch", "Hq", "Hkv", "N", "d",
+             "B", "max_sel", "scale", "dQ", "dK", "dV", "delta", "stream"]
+    ok = [FAKE] * 6 + [1, FAKE, FAKE, 1, 8, 2, 4096, 128, 64, 18, 0.088, FAKE, FAKE, FAKE, FAKE,
+                       NULL]
+
+    def call(**kw):
+        args = list(ok)
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return fn(*args)
+
+    assert call(dt=0) == 2                   # fp32: not implemented
+    assert call(dt=7) == 1                   # unknown dtype
+    assert call(d=96) == 2
+    assert call(B=40) == 2
+    assert call(Hq=6, Hkv=4) == 1            # Hq not a multiple of Hkv
+    assert call(N=0) == 1
+    assert call(max_sel=0) == 1
+    assert call(scale=0.0) == 1
+    for name in ("Q", "K", "V", "O", "dO", "lse", "idx", "cnt", "dQ", "dK", "dV", "delta"):
+        assert call(**{name: NULL}) == 1, name
+    assert call(dK=ctypes.c_void_p(0x100008)) == 1  # not 16-byte aligned
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(ImportError):
         abi.load_library(str(tmp_path / "missing.so"))

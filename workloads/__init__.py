@@ -33,6 +33,7 @@ __all__ = [
     "CONFIGS",
     "planted_prefill",
     "planted_decode",
+    "upstream_grad",
     "to_f64",
 ]
 
@@ -160,6 +161,14 @@ def planted_decode(batch, Hq, Hkv, Lmax, d, B, clusters, seed=0, dtype="bf16",
         seqlens = torch.full((batch,), Lmax, dtype=torch.int32)
     seqlens = torch.as_tensor(seqlens, dtype=torch.int32).to(device)
     return q.to(t).contiguous(), Kc, Vc, seqlens
+
+
+def upstream_grad(batch, Hq, N, d, seed=0, dtype="bf16", device="cpu"):
+    """Gradient of a loss with respect to the attention output: ``[batch, Hq, N, d]``
+    standard normal entries (the backward pass's ``dO``)."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    g = torch.randn(batch, Hq, N, d, generator=gen, device=device)
+    return g.to(_torch_dtype(dtype)).contiguous()
 
 
 def to_f64(x) -> np.ndarray:
