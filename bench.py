@@ -16,6 +16,11 @@ beside it.  Inputs are seeded synthetic tensors (planted clusters) resident in
 HBM; the working sets exceed the 126 MB L2 (Q alone is 256 MiB, a decode step
 reads ~840 MB), so no flush is done between steps.
 
+Two calls are timed apart from the step and reported under `kernels`: the
+decode-cache append (a CUDA graph of 20 calls, every append completing a
+block) and the backward of the prefill attention on the step's own selection
+(8 * d FLOPs per unmasked pair: the dV, dP, dQ and dK contractions).
+
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same
 workload instead (there is no runnable upstream implementation).
 """
