@@ -16,3 +16,9 @@ from .ssa_oracle import (  # noqa: F401
     sparse_attention_backward,
     summary_scores,
 )
+from .dash_oracle import (  # noqa: F401
+    entmax,
+    entmax_route,
+    learned_block_summary,
+    prior_sparse_attention,
+)
