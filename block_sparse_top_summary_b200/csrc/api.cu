@@ -36,7 +36,7 @@ const char* ssa_status_string(int status) {
   }
 }
 
-int ssa_version(void) { return 100; }
+int ssa_version(void) { return 102; }
 
 ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv, int N, int d,
                              int B, float* S, ssa_stream stream) {

@@ -55,7 +55,8 @@ typedef struct CUstream_st* ssa_stream;
 /* Human-readable name of a status code.  Never NULL. */
 const char* ssa_status_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor).  1.01 added ssa_decode_append,
+ * 1.02 ssa_sparse_attn_bwd. */
 int ssa_version(void);
 
 /*

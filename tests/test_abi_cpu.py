@@ -42,7 +42,7 @@ def test_status_strings_and_version(lib):
     assert lib.ssa_status_string(0) == b"SSA_OK"
     assert lib.ssa_status_string(4) == b"SSA_ERR_TIMEOUT"
     assert lib.ssa_status_string(99) == b"SSA_ERR_UNKNOWN"
-    assert lib.ssa_version() >= 100
+    assert lib.ssa_version() >= 102
 
 
 NULL = None
