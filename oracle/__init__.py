@@ -22,3 +22,9 @@ from .dash_oracle import (  # noqa: F401
     learned_block_summary,
     prior_sparse_attention,
 )
+from .hier_oracle import (  # noqa: F401
+    decode_per_head,
+    decode_route_per_head,
+    hierarchical_route,
+    segment_summaries,
+)
