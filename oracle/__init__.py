@@ -28,3 +28,8 @@ from .hier_oracle import (  # noqa: F401
     hierarchical_route,
     segment_summaries,
 )
+from .paged_oracle import (  # noqa: F401
+    decode_append_paged,
+    decode_paged,
+    gather_pages,
+)
