@@ -1,0 +1,27 @@
+"""The benchmark's work accounting against an independent count.
+
+``bench.attn_flops`` counts 4 d FLOPs per unmasked (query, key) pair of the
+selected blocks from the routing counts alone.  The oracle's attention matrix
+P has a positive entry exactly for every such pair, so counting them is an
+independent check, including the ragged last block and GQA groups.
+"""
+import numpy as np
+import pytest
+
+import bench
+import oracle as O
+
+
+@pytest.mark.parametrize("N,B,topk,Hq,Hkv", [(8 * 9 + 3, 8, 2, 4, 2), (16 * 6, 16, 1, 2, 1),
+                                            (8 * 7 + 5, 8, 100, 3, 1)])
+def test_attn_flops_counts_every_attended_pair(N, B, topk, Hq, Hkv):
+    rng = np.random.default_rng(N + topk)
+    d = 8
+    Q = rng.standard_normal((1, Hq, N, d))
+    K = rng.standard_normal((1, Hkv, N, d))
+    idx, cnt, _ = O.route(Q, O.block_summary(K, B), B, topk, Hkv)
+    P = O.attention_probs(Q, K, idx, cnt, B)
+    pairs = int(np.count_nonzero(P > 0))
+    G = Hq // Hkv
+    flops = sum(bench.attn_flops(cnt[0, g], N, B, G, d) for g in range(Hkv))
+    assert flops == pairs * 4 * d
