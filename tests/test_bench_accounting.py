@@ -25,3 +25,25 @@ def test_attn_flops_counts_every_attended_pair(N, B, topk, Hq, Hkv):
     G = Hq // Hkv
     flops = sum(bench.attn_flops(cnt[0, g], N, B, G, d) for g in range(Hkv))
     assert flops == pairs * 4 * d
+
+
+def test_decode_bytes_counts_the_rows_each_selection_reads():
+    # K and V rows = cache positions t < L whose block is selected; summaries =
+    # the complete candidate blocks 1 .. last-1 (fp32); plus q and O
+    rng = np.random.default_rng(5)
+    batch, Hq, Hkv, Lmax, d, B, topk = 3, 4, 2, 8 * 10, 8, 8, 3
+    q = rng.standard_normal((batch, Hq, d))
+    Kc = rng.standard_normal((batch, Hkv, Lmax, d))
+    L = np.array([80, 43, 1])
+    S = np.stack([O.block_summary(Kc[b : b + 1], B)[0] for b in range(batch)])
+    idx, cnt, _ = O.decode_route(q, S, L, B, topk)
+    esize = 2
+    expect = 0.0
+    for b in range(batch):
+        last = (L[b] - 1) // B
+        for g in range(Hkv):
+            sel = set(int(j) for j in idx[b, g, : cnt[b, g]])
+            rows = sum(1 for t in range(L[b]) if t // B in sel)
+            expect += 2 * rows * d * esize + len(range(1, max(last, 1))) * d * 4
+    expect += 2 * batch * Hq * d * esize
+    assert bench.decode_bytes(idx, L, B, d, Hq // Hkv, esize) == expect
