@@ -30,7 +30,13 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(
   constexpr int CPR = D / EPC;      // chunks per row
   const int b = blockIdx.x;
   const int t = threadIdx.x;
-  const int L = seqlens[b];
+  // Thread 0 reads the length once and shares it: thread 0 raises seqlens[b]
+  // at the end, and a warp that read it directly after that store would take
+  // the new length for the old one.
+  __shared__ int s_len;
+  if (t == 0) s_len = seqlens[b];
+  __syncthreads();
+  const int L = s_len;
   if (L < 0 || L >= Lmax) return;  // full cache or invalid length: nothing changes
   const int64_t head0 = (int64_t)b * Hkv;
   // the new rows: chunk w of head h (w < CPR: key, else value)

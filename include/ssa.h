@@ -242,7 +242,10 @@ ssa_status ssa_decode_append(void* Kc, void* Vc, ssa_dtype dtype, float* S, int3
  * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  * - The first call on each device looks up that device's address of the array
  *   (with the device current), so make that first call before any stream
- *   capture; later calls only read the cached address.
+ *   capture; later calls only read the cached address.  The cached address
+ *   belongs to the device's primary context as it was at that first call: after
+ *   cudaDeviceReset on that device it is stale, so do not call this entry point
+ *   on a device that was reset after its first call.
  * - All calls share the one array and it keeps the previous call's contents;
  *   everything that must start at zero is cleared by the call itself.  Calls
  *   that overlap on the GPU (other streams, other host threads) race on it:

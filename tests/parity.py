@@ -67,3 +67,14 @@ def out_errors(gpu, ref):
     den = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(diff) / den) if den > 0 else float(np.linalg.norm(diff))
     return max_abs, rel
+
+
+# Per-workload parity counts of this test session (selection rows, near-ties,
+# mismatches, output errors), printed at the end of the run by conftest.py.
+REPORT: dict = {}
+
+
+def record(name: str, doc: dict):
+    """Add one workload's parity counts to the session report."""
+    REPORT[name] = doc
+    print(name, doc)

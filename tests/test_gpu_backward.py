@@ -1,12 +1,19 @@
 """GPU-vs-oracle parity of the backward pass of the selected-block attention.
 
 Both sides take the oracle's selection, so routing plays no part.  The GPU
-backward gets the GPU forward's O (bf16) and log-sum-exp.  Tolerance for the
-bf16 gradients, per tensor: relative-L2 <= 1e-2 and max-abs <= 2e-2 of the
-reference's largest magnitude.  The kernel rounds P and dS to bf16 as mma
-operands and every output to bf16 (each 2^-9 relative), and delta uses the
-bf16 O, so errors of a few 1e-3 relative are expected; the bounds leave a
-margin of about 3.
+backward gets the GPU forward's O (bf16) and log-sum-exp.
+
+Tolerance, per gradient tensor: the bf16 bounds that hold for every output of
+this library, relative-L2 <= 5e-3 and max-abs <= 2e-2.  An absolute bound only
+means something on values of a known scale, so the upstream gradient dO is
+drawn with standard deviation 1/4: every gradient then stays below 4 in
+magnitude (the largest over these cases is about 2.3), where one bf16
+rounding of an output costs at most half an ulp, 2^-7 = 0.0078.  (With dO of
+standard deviation 1 the gradients reach 9, and a single bf16 rounding there
+is already 0.031.)  The kernel also rounds P and dS to bf16 as mma operands
+(2^-9 relative each) and forms delta from the bf16 O; the relative-L2 error
+this gives is about 2.6e-3.  A max-abs bound relative to the tensor's largest
+magnitude (2e-2) is kept as an extra check.
 """
 import numpy as np
 import pytest
@@ -20,8 +27,10 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 DEV = "cuda"
-REL_L2 = 1e-2
+REL_L2 = 5e-3      # bf16 relative-L2 bound
+MAX_ABS = 2e-2     # bf16 max-abs bound
 MAX_ABS_REL = 2e-2
+DO_STD = 0.25      # standard deviation of the upstream gradient
 
 
 @pytest.fixture(scope="module")
@@ -33,7 +42,7 @@ def ssa():
 
 def _case(ssa, batch, Hq, Hkv, N, d, B, topk, clusters, seed):
     Q, K, V = planted_prefill(batch, Hq, Hkv, N, d, B, clusters, seed=seed, dtype="bf16")
-    dO = upstream_grad(batch, Hq, N, d, seed=seed + 100, dtype="bf16")
+    dO = upstream_grad(batch, Hq, N, d, seed=seed + 100, dtype="bf16", std=DO_STD)
     Qf, Kf, Vf, dOf = (to_f64(x) for x in (Q, K, V, dO))
     idx, cnt, _ = O.route(Qf, O.block_summary(Kf, B), B, topk, Hkv)
     gi = torch.from_numpy(idx.astype(np.int32)).to(DEV)
@@ -53,7 +62,9 @@ def _check(gpu, ref):
         assert np.all(np.isfinite(g)), name
         ma, rel = out_errors(g, r)
         scale = float(np.max(np.abs(r)))
-        assert rel <= REL_L2 and ma <= MAX_ABS_REL * scale, (name, ma, scale, rel)
+        assert scale < 4.0, (name, scale)  # the range the absolute bound is stated for
+        assert rel <= REL_L2 and ma <= MAX_ABS, (name, ma, rel)
+        assert ma <= MAX_ABS_REL * scale, (name, ma, scale)
 
 
 @pytest.mark.parametrize("batch,Hq,Hkv,N,d,B,topk,clusters", [

@@ -312,6 +312,30 @@ def test_decode_append_parity(ssa, dtype, d, B):
     assert np.array_equal(got[~changed], S.double().numpy()[~changed])  # the rest untouched, bitwise
 
 
+def test_decode_append_many_in_a_row_narrow_cache(ssa):
+    # One KV head with d = 64 in bf16 keeps 16 of the CTA's 1024 threads busy
+    # copying rows, so most warps read the length long after thread 0 could
+    # have raised it.  200 appends in a row, nearly all of them ending
+    # mid-block, must give the oracle's cache, summaries and lengths.
+    B, d, batch, Hkv, Lmax = 64, 64, 3, 1, 64 * 5
+    gen = torch.Generator().manual_seed(41)
+    Kc = torch.zeros(batch, Hkv, Lmax, d).to(torch.bfloat16)
+    Vc = torch.zeros(batch, Hkv, Lmax, d).to(torch.bfloat16)
+    S = torch.zeros(batch, Hkv, Lmax // B, d)
+    L = torch.tensor([0, 37, 250], dtype=torch.int32)
+    Kd, Vd, Sd, Ld = Kc.to(DEV), Vc.to(DEV), S.to(DEV), L.to(DEV)
+    rK, rV, rS, rL = to_f64(Kc), to_f64(Vc), S.double().numpy(), L.numpy()
+    for _ in range(200):
+        kn = torch.randn(batch, Hkv, d, generator=gen).to(torch.bfloat16)
+        vn = torch.randn(batch, Hkv, d, generator=gen).to(torch.bfloat16)
+        ssa.ssa_decode_append(Kd, Vd, Sd, Ld, kn.to(DEV), vn.to(DEV), B)
+        rK, rV, rS, rL = O.decode_append(rK, rV, rS, rL, to_f64(kn), to_f64(vn), B)
+    torch.cuda.synchronize()
+    assert Ld.cpu().tolist() == rL.tolist() == [200, 237, Lmax]
+    assert np.array_equal(to_f64(Kd.cpu()), rK) and np.array_equal(to_f64(Vd.cpu()), rV)
+    np.testing.assert_allclose(Sd.cpu().double().numpy(), rS, rtol=0, atol=F32_MAX_ABS)
+
+
 def test_append_then_decode_matches_oracle(ssa):
     # A serving loop: three appends, one of which completes a block, then one
     # decode step on the grown caches.

@@ -163,11 +163,13 @@ def planted_decode(batch, Hq, Hkv, Lmax, d, B, clusters, seed=0, dtype="bf16",
     return q.to(t).contiguous(), Kc, Vc, seqlens
 
 
-def upstream_grad(batch, Hq, N, d, seed=0, dtype="bf16", device="cpu"):
+def upstream_grad(batch, Hq, N, d, seed=0, dtype="bf16", device="cpu", std=1.0):
     """Gradient of a loss with respect to the attention output: ``[batch, Hq, N, d]``
-    standard normal entries (the backward pass's ``dO``)."""
+    normal entries of standard deviation ``std`` (the backward pass's ``dO``)."""
     gen = torch.Generator(device=device).manual_seed(seed)
     g = torch.randn(batch, Hq, N, d, generator=gen, device=device)
+    if std != 1.0:
+        g = g * std
     return g.to(_torch_dtype(dtype)).contiguous()
 
 
