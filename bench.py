@@ -1,25 +1,36 @@
 """Benchmark of the block-sparse attention hot path on B200.
 
 One step = one pass of the whole hot path:
-  prefill on the 32K workload (1 x 32 query heads / 8 KV heads, N = 32768,
-  d = 128, bf16, B = 64, top-k = 16 + sink + diagonal):
+  prefill on the headline workload, by default the 128K one (1 x 32 query
+  heads / 8 KV heads, N = 131072, d = 128, bf16, B = 64, top-k = 32 + sink +
+  diagonal):
       ssa_block_summary -> ssa_route -> ssa_sparse_attn_fwd
   followed by one decode step on the decode workload (64 sequences x 65536
   cached tokens, 32 / 8 heads, d = 128, bf16, B = 64, top-k = 32 + sink + last):
       ssa_decode (route + split-KV attention + log-sum-exp combine).
+`--workload prefill32k` makes the 32K workload (N = 32768, top-k = 16) the
+step's prefill instead.
 
 `value` is the prefill selected-block TFLOP/s: algorithmic FLOPs of the
 attention (4 * d per unmasked (query, key) pair of the selected blocks,
 counted from the routing output) over the device time of the prefill pass
 (summary + route + attention).  Decode tokens/s and HBM GB/s are reported
-beside it.  Inputs are seeded synthetic tensors (planted clusters) resident in
-HBM; the working sets exceed the 126 MB L2 (Q alone is 256 MiB, a decode step
-reads ~840 MB), so no flush is done between steps.
+beside it.  Inputs are seeded synthetic tensors (planted clusters) drawn on
+the device and resident in HBM; the working sets exceed the 126 MB L2 (Q
+alone is 1 GiB at 128K, a decode step reads ~840 MB), so no flush is done
+between steps.
 
-Two calls are timed apart from the step and reported under `kernels`: the
-decode-cache append (a CUDA graph of 20 calls, every append completing a
-block) and the backward of the prefill attention on the step's own selection
-(8 * d FLOPs per unmasked pair: the dV, dP, dQ and dK contractions).
+Timed apart from the step and reported under their own keys:
+- `prefill32k`: the prefill pass on the other prefill workload;
+- `sweep`: the sparsity sweep (2 x 16 / 4 heads, N = 65536, B = 128) at
+  top-k = 4, 8, 16, 32, 64 and all: attention TFLOP/s against k;
+- `kernels.ssa_decode_append`: the decode-cache append (a CUDA graph of 20
+  calls, every append completing a block);
+- `kernels.ssa_sparse_attn_bwd`: the backward of the 32K prefill attention on
+  its own selection (8 * d FLOPs per unmasked pair: the dV, dP, dQ and dK
+  contractions).
+Every kernel line carries its fraction of the measured peak (MEASURED_PEAKS)
+and of the nominal one (2.25 PFLOP/s dense bf16, 8 TB/s HBM).
 
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same
 workload instead (there is no runnable upstream implementation).
@@ -39,9 +50,13 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import CONFIGS, planted_decode, planted_prefill, upstream_grad  # noqa: E402
+from workloads import CONFIGS, TOPK_ALL, planted_decode, planted_prefill, upstream_grad  # noqa: E402
 
 METRIC = "prefill selected-block TFLOP/s & % BF16 peak; decode tokens/s & HBM GB/s"
+
+# Nominal B200 peaks the targets are stated against.
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
 
 
 # ------------------------------------------------------------- work accounting
@@ -69,12 +84,12 @@ def decode_bytes(idx: np.ndarray, seqlens: np.ndarray, B: int, d: int, G: int, e
     return total
 
 
-def attn_traffic_per_launch():
-    """DRAM bytes (read + write) per attention launch from the committed ncu
-    record, or None when the kernel source changed since the capture."""
+def traffic_per_launch(record: str, source: str):
+    """DRAM bytes (read + write) per launch from a committed ncu record under
+    profiles/, or None when the kernel source changed since the capture."""
     import hashlib
-    rec = os.path.join(ROOT, "profiles", "attn_tc_prefill32k_traffic.txt")
-    src = os.path.join(ROOT, "block_sparse_top_summary_b200", "csrc", "attn_tc.cu")
+    rec = os.path.join(ROOT, "profiles", record)
+    src = os.path.join(ROOT, "block_sparse_top_summary_b200", "csrc", source)
     if not (os.path.exists(rec) and os.path.exists(src)):
         return None
     kv = {}
@@ -199,55 +214,140 @@ def sum_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def fracs(achieved: float, measured: float, nominal: float) -> dict:
+    """Fractions of the measured and of the nominal peak."""
+    return {"frac": achieved / measured, "frac_nominal": achieved / nominal}
+
+
+def describe(c, topk=None) -> str:
+    """The workload's name and sizes (`topk` overrides its top-k; a string is
+    printed as is)."""
+    k = c.topk if topk is None else topk
+    k = "all" if not isinstance(k, str) and k >= TOPK_ALL else k
+    return (f"{c.name} ({c.batch}x{c.Hq}q/{c.Hkv}kv, N={c.N}, d={c.d}, {c.dtype}, B={c.B}, "
+            f"top-k={k})")
+
+
 # ------------------------------------------------------------- our arm
+class Prefill:
+    """Device buffers and the three prefill calls of one prefill workload."""
+
+    def __init__(self, ssa, c, dev, seed, topk=None):
+        self.ssa, self.c = ssa, c
+        self.topk = c.topk if topk is None else topk
+        self.Q, self.K, self.V = planted_prefill(c.batch, c.Hq, c.Hkv, c.N, c.d, c.B, c.clusters,
+                                                 seed=seed, dtype=c.dtype, device=dev)
+        nq = -(-c.N // c.B)
+        self.max_sel = ssa.route_width(c.N, c.B, self.topk)
+        self.S = torch.empty(c.batch, c.Hkv, c.N // c.B, c.d, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(c.batch, c.Hkv, nq, self.max_sel, dtype=torch.int32, device=dev)
+        self.cnt = torch.empty(c.batch, c.Hkv, nq, dtype=torch.int32, device=dev)
+        self.O = torch.empty_like(self.Q)
+        self.lse = torch.empty(c.batch, c.Hq, c.N, dtype=torch.float32, device=dev)
+
+    def set_topk(self, topk):
+        c = self.c
+        self.topk = topk
+        nq = -(-c.N // c.B)
+        self.max_sel = self.ssa.route_width(c.N, c.B, topk)
+        self.idx = torch.empty(c.batch, c.Hkv, nq, self.max_sel, dtype=torch.int32,
+                               device=self.Q.device)
+
+    def run(self, evs=None, stream=None):
+        ssa, c = self.ssa, self.c
+        if evs:
+            evs[0].record(stream)
+        ssa.ssa_block_summary(self.K, c.B, S=self.S)
+        if evs:
+            evs[1].record(stream)
+        ssa.ssa_route(self.Q, self.S, c.B, self.topk, c.Hkv, max_sel=self.max_sel, idx=self.idx,
+                      cnt=self.cnt)
+        if evs:
+            evs[2].record(stream)
+        ssa.ssa_sparse_attn_fwd(self.Q, self.K, self.V, self.idx, self.cnt, c.B, O=self.O,
+                                lse=self.lse)
+        if evs:
+            evs[3].record(stream)
+
+    def flops(self):
+        c = self.c
+        cnt = self.cnt.cpu().numpy()
+        return sum(attn_flops(cnt[b, g], c.N, c.B, c.Hq // c.Hkv, c.d)
+                   for b in range(c.batch) for g in range(c.Hkv))
+
+    def summary_bytes(self):
+        return self.K.numel() * self.K.element_size() + self.S.numel() * 4
+
+    def route_bytes(self):
+        return (self.Q.numel() * self.Q.element_size() + self.S.numel() * 4 +
+                self.idx.numel() * 4 + self.cnt.numel() * 4)
+
+
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def time_prefill(p: Prefill, iters: int, warmup: int, stream, world):
+    """Mean per-call device times (ms) of summary, route and attention."""
+    for _ in range(warmup):
+        p.run()
+    torch.cuda.synchronize()
+    evs = [[_ev() for _ in range(4)] for _ in range(iters)]
+    barrier(world)
+    for k in range(iters):
+        p.run(evs[k], stream)
+    torch.cuda.synchronize()
+    seg = np.array([[evs[k][s].elapsed_time(evs[k][s + 1]) for s in range(3)]
+                    for k in range(iters)])
+    return [max_over_ranks(float(x), world) for x in seg.mean(axis=0)]
+
+
+def prefill_report(p: Prefill, seg, flops, hbm_peak, bf16_peak, tc):
+    sm, rt, at = seg
+    pass_ms = sm + rt + at
+    att = flops / (at * 1e-3) / 1e12
+    sgb = p.summary_bytes() / (sm * 1e-3) / 1e9
+    rgb = p.route_bytes() / (rt * 1e-3) / 1e9
+    return {
+        "workload": describe(p.c, p.topk),
+        "pass_ms": pass_ms, "TFLOP/s": flops / (pass_ms * 1e-3) / 1e12,
+        "attn_flops": flops,
+        "ssa_block_summary": {"ms": sm, "bound": "hbm", "GB/s": sgb,
+                              **fracs(sgb, hbm_peak, NOMINAL_HBM_GBS),
+                              "bytes": p.summary_bytes()},
+        "ssa_route": {"ms": rt, "bound": "hbm", "GB/s": rgb,
+                      **fracs(rgb, hbm_peak, NOMINAL_HBM_GBS), "bytes": p.route_bytes()},
+        "ssa_sparse_attn_fwd": {"ms": at, "bound": "tensor" if tc else "alu", "TFLOP/s": att,
+                                **fracs(att, bf16_peak, NOMINAL_BF16_TFLOPS)},
+    }
+
+
 def run_ours(args, world, rank, local):
     import block_sparse_top_summary_b200 as ssa
     ssa.load_library()
     dev = torch.device("cuda", local)
     hbm_peak, bf16_peak, peak_kind = load_peaks()
-    cp = CONFIGS["prefill32k"]
+    head = args.workload
+    other = "prefill32k" if head == "prefill128k" else "prefill128k"
+    cp = CONFIGS[head]
     cd = CONFIGS["decode"]
-    G = cp.Hq // cp.Hkv
+    stream = torch.cuda.current_stream(dev)
 
-    # --- inputs (seed offset by rank: each rank works on its own problem)
-    Q, K, V = planted_prefill(cp.batch, cp.Hq, cp.Hkv, cp.N, cp.d, cp.B, cp.clusters,
-                              seed=rank_seed(cp.seed, rank), dtype=cp.dtype)
-    Qh, Kh, Vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
-    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    # --- inputs, drawn on the device (seed offset by rank: each rank works on
+    # its own problem)
+    P = Prefill(ssa, cp, dev, rank_seed(cp.seed, rank))
     q, Kc, Vc, L = planted_decode(cd.batch, cd.Hq, cd.Hkv, cd.L, cd.d, cd.B, cd.clusters,
                                   seed=rank_seed(cd.seed, rank), dtype=cd.dtype, device=dev)
     Sc = ssa.ssa_block_summary(Kc, cd.B)  # precomputed cache summaries (decode input)
-    qh, Lh = q.cpu().pin_memory(), L.cpu().pin_memory()
-
-    stream = torch.cuda.current_stream(dev)
-    nq = -(-cp.N // cp.B)
-    max_sel = ssa.route_width(cp.N, cp.B, cp.topk)
-    S = torch.empty(cp.batch, cp.Hkv, cp.N // cp.B, cp.d, dtype=torch.float32, device=dev)
-    idx = torch.empty(cp.batch, cp.Hkv, nq, max_sel, dtype=torch.int32, device=dev)
-    cnt = torch.empty(cp.batch, cp.Hkv, nq, dtype=torch.int32, device=dev)
-    Od = torch.empty_like(Qd)
-    lse = torch.empty(cp.batch, cp.Hq, cp.N, dtype=torch.float32, device=dev)
     Odec = torch.empty_like(q)
     didx = torch.empty(cd.batch, cd.Hkv, ssa.decode_width(cd.L, cd.B, cd.topk), dtype=torch.int32,
                        device=dev)
     ws = torch.empty(ssa.ssa_decode_workspace_size(cd.batch, cd.Hq, cd.Hkv, cd.L, cd.d, cd.B,
                                                    cd.topk), dtype=torch.uint8, device=dev)
-
-    def ev():
-        return torch.cuda.Event(enable_timing=True)
+    G = cp.Hq // cp.Hkv
 
     def step(evs=None):
-        if evs:
-            evs[0].record(stream)
-        ssa.ssa_block_summary(Kd, cp.B, S=S)
-        if evs:
-            evs[1].record(stream)
-        ssa.ssa_route(Qd, S, cp.B, cp.topk, cp.Hkv, max_sel=max_sel, idx=idx, cnt=cnt)
-        if evs:
-            evs[2].record(stream)
-        ssa.ssa_sparse_attn_fwd(Qd, Kd, Vd, idx, cnt, cp.B, O=Od, lse=lse)
-        if evs:
-            evs[3].record(stream)
+        P.run(evs, stream)
         ssa.ssa_decode(q, Kc, Vc, Sc, L, cd.B, cd.topk, O=Odec, idx=didx, workspace=ws)
         if evs:
             evs[4].record(stream)
@@ -255,17 +355,16 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    flops = attn_flops(cnt[0].cpu().numpy(), cp.N, cp.B, G, cp.d) * cp.batch
+    assert ssa.ssa_device_error() == 0
+    flops = P.flops()
     dbytes = decode_bytes(didx.cpu().numpy(), L.cpu().numpy(), cd.B, cd.d, cd.Hq // cd.Hkv, 2)
-    sum_bytes = K.numel() * 2 + S.numel() * 4
-    route_bytes = Q.numel() * 2 + S.numel() * 4 + idx.numel() * 4 + cnt.numel() * 4
 
     clocks = ClockSampler(torch.cuda.current_device())
-    evs = [[ev() for _ in range(5)] for _ in range(args.steps)]
+    evs = [[_ev() for _ in range(5)] for _ in range(args.steps)]
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
-    t0, t1 = ev(), ev()
+    t0, t1 = _ev(), _ev()
     t0.record(stream)
     for k in range(args.steps):
         step(evs[k])
@@ -276,29 +375,35 @@ def run_ours(args, world, rank, local):
     total_ms = max_over_ranks(t0.elapsed_time(t1), world)
     seg = np.array([[evs[k][s].elapsed_time(evs[k][s + 1]) for s in range(4)]
                     for k in range(args.steps)])  # ms: summary, route, attn, decode
-    seg_mean = seg.mean(axis=0)
+    seg_mean = [max_over_ranks(float(x), world) for x in seg.mean(axis=0)]
     prefill_ms = max_over_ranks(float(seg[:, :3].sum(axis=1).mean()), world)
-    decode_ms = max_over_ranks(float(seg_mean[3]), world)
-    attn_ms = float(seg_mean[2])
+    decode_ms = seg_mean[3]
 
     all_flops = sum_over_ranks(flops, world)
     value = all_flops / (prefill_ms * 1e-3) / 1e12
-    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    tc = ssa.ssa_sparse_attn_uses_tensor_cores(torch.bfloat16, cp.Hq, cp.Hkv, cp.d, cp.B)
+    head_rep = prefill_report(P, seg_mean[:3], flops, hbm_peak, bf16_peak, tc)
+    attn_tflops = head_rep["ssa_sparse_attn_fwd"]["TFLOP/s"]
     dec_tok = sum_over_ranks(cd.batch, world) / (decode_ms * 1e-3)
     dec_gbs = dbytes / (decode_ms * 1e-3) / 1e9
 
-    # --- end to end through the C ABI from pinned host buffers
+    # --- end to end through the C ABI from pinned host buffers: the step's
+    # prefill inputs and decode query in, both outputs out, every step
+    Qh = P.Q.cpu().pin_memory()
+    Kh = P.K.cpu().pin_memory()
+    Vh = P.V.cpu().pin_memory()
+    qh, Lh = q.cpu().pin_memory(), L.cpu().pin_memory()
     Oh = torch.empty_like(Qh).pin_memory()
     Odh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
 
     def e2e_step():
-        Qd.copy_(Qh, non_blocking=True)
-        Kd.copy_(Kh, non_blocking=True)
-        Vd.copy_(Vh, non_blocking=True)
+        P.Q.copy_(Qh, non_blocking=True)
+        P.K.copy_(Kh, non_blocking=True)
+        P.V.copy_(Vh, non_blocking=True)
         q.copy_(qh, non_blocking=True)
         L.copy_(Lh, non_blocking=True)
         step()
-        Oh.copy_(Od, non_blocking=True)
+        Oh.copy_(P.O, non_blocking=True)
         Odh.copy_(Odec, non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 5))
@@ -306,26 +411,56 @@ def run_ours(args, world, rank, local):
         e2e_step()
     torch.cuda.synchronize()
     barrier(world)
-    a, b_ = ev(), ev()
+    a, b_ = _ev(), _ev()
     a.record(stream)
     for _ in range(e2e_steps):
         e2e_step()
     b_.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a.elapsed_time(b_) / e2e_steps, world)
-    h2d = (Q.numel() + K.numel() + V.numel() + q.numel()) * 2 + L.numel() * 4
-    d2h = Q.numel() * 2 + q.numel() * 2
+    h2d = (Qh.numel() + Kh.numel() + Vh.numel() + qh.numel()) * 2 + Lh.numel() * 4
+    d2h = Oh.numel() * 2 + Odh.numel() * 2
+    del Qh, Kh, Vh, Oh
+
+    # --- the other prefill workload, timed apart
+    po = Prefill(ssa, CONFIGS[other], dev, rank_seed(CONFIGS[other].seed, rank))
+    seg_o = time_prefill(po, iters=10, warmup=3, stream=stream, world=world)
+    other_rep = prefill_report(po, seg_o, po.flops(), hbm_peak, bf16_peak,
+                               ssa.ssa_sparse_attn_uses_tensor_cores(
+                                   torch.bfloat16, po.c.Hq, po.c.Hkv, po.c.d, po.c.B))
+    p32 = P if head == "prefill32k" else po  # the backward runs on the 32K workload
+    if head == "prefill32k":
+        del po
+
+    # --- the sparsity sweep: attention TFLOP/s against k, "all" last
+    cs = CONFIGS["sweep"]
+    ps = Prefill(ssa, cs, dev, rank_seed(cs.seed, rank))
+    sweep = []
+    for k in cs.topk_sweep:
+        ps.set_topk(k)
+        seg_s = time_prefill(ps, iters=5 if k >= TOPK_ALL else 10, warmup=3, stream=stream,
+                             world=world)
+        rep = prefill_report(ps, seg_s, ps.flops(), hbm_peak, bf16_peak,
+                             ssa.ssa_sparse_attn_uses_tensor_cores(torch.bfloat16, cs.Hq, cs.Hkv,
+                                                                   cs.d, cs.B))
+        sweep.append({"topk": "all" if k >= TOPK_ALL else k, "attn_flops": rep["attn_flops"],
+                      "attn_ms": rep["ssa_sparse_attn_fwd"]["ms"],
+                      "attn_TFLOP/s": rep["ssa_sparse_attn_fwd"]["TFLOP/s"],
+                      "attn_frac": rep["ssa_sparse_attn_fwd"]["frac"],
+                      "attn_frac_nominal": rep["ssa_sparse_attn_fwd"]["frac_nominal"],
+                      "pass_ms": rep["pass_ms"], "pass_TFLOP/s": rep["TFLOP/s"]})
+    del ps
 
     # --- appending one token per sequence (incremental decoding), timed on its
-    # own after everything else, as it rewrites a cache row.  Every call is
-    # set up so that its append completes a block (the costlier case): 20
-    # calls, each with its own copy of the lengths, are captured in a CUDA graph
-    # and replayed, so the device time carries no host gaps; the lengths are
+    # own after the step, as it rewrites a cache row.  Every call is set up so
+    # that its append completes a block (the costlier case): 20 calls, each
+    # with its own copy of the lengths, are captured in a CUDA graph and
+    # replayed, so the device time carries no host gaps; the lengths are
     # restored between replays, outside the timed events.
     app_len = torch.full_like(L, (cd.L // cd.B - 1) * cd.B - 1)
     app_Ls = [app_len.clone() for _ in range(20)]
-    kn = torch.randn(cd.batch, cd.Hkv, cd.d, device=q.device).to(torch.bfloat16)
-    vn = torch.randn(cd.batch, cd.Hkv, cd.d, device=q.device).to(torch.bfloat16)
+    kn = torch.randn(cd.batch, cd.Hkv, cd.d, device=dev).to(torch.bfloat16)
+    vn = torch.randn(cd.batch, cd.Hkv, cd.d, device=dev).to(torch.bfloat16)
     ssa.ssa_decode_append(Kc, Vc, Sc, app_Ls[0], kn, vn, cd.B, stream=stream)  # warm-up
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
@@ -337,7 +472,7 @@ def run_ours(args, world, rank, local):
         for t_ in app_Ls:
             t_.copy_(app_len)
         torch.cuda.synchronize()
-        a, b_ = ev(), ev()
+        a, b_ = _ev(), _ev()
         a.record(stream)
         graph.replay()
         b_.record(stream)
@@ -349,21 +484,24 @@ def run_ours(args, world, rank, local):
     # per sequence and KV head: two rows written, the completed block's B key rows
     # read back, one fp32 summary row written
     app_bytes = cd.batch * cd.Hkv * (2 * cd.d * 2 + cd.B * cd.d * 2 + cd.d * 4)
+    app_gbs = app_bytes / (app_ms * 1e-3) / 1e9
 
-    # --- backward of the attention (training), timed apart from the step on the
-    # step's own selection, O and log-sum-exp
-    dOd = upstream_grad(cp.batch, cp.Hq, cp.N, cp.d, seed=rank_seed(cp.seed + 1, rank),
-                        dtype=cp.dtype, device=dev)
-    dQb, dKb, dVb = torch.empty_like(Qd), torch.empty_like(Kd), torch.empty_like(Vd)
-    delta = torch.empty(cp.batch, cp.Hq, cp.N, dtype=torch.float32, device=dev)
+    # --- backward of the 32K attention (training), timed apart from the step
+    # on that workload's own selection, O and log-sum-exp
+    c32 = p32.c
+    p32.run()
+    dOd = upstream_grad(c32.batch, c32.Hq, c32.N, c32.d, seed=rank_seed(c32.seed + 1, rank),
+                        dtype=c32.dtype, device=dev)
+    dQb, dKb, dVb = torch.empty_like(p32.Q), torch.empty_like(p32.K), torch.empty_like(p32.V)
+    delta = torch.empty(c32.batch, c32.Hq, c32.N, dtype=torch.float32, device=dev)
 
     def bwd():
-        ssa.ssa_sparse_attn_bwd(Qd, Kd, Vd, Od, dOd, lse, idx, cnt, cp.B, dQ=dQb, dK=dKb, dV=dVb,
-                                delta=delta)
+        ssa.ssa_sparse_attn_bwd(p32.Q, p32.K, p32.V, p32.O, dOd, p32.lse, p32.idx, p32.cnt,
+                                c32.B, dQ=dQb, dK=dKb, dV=dVb, delta=delta)
 
     bwd_ms = []
     for it in range(2 + 5):
-        a, b_ = ev(), ev()
+        a, b_ = _ev(), _ev()
         a.record(stream)
         bwd()
         b_.record(stream)
@@ -372,60 +510,58 @@ def run_ours(args, world, rank, local):
             bwd_ms.append(a.elapsed_time(b_))
     bwd_ms = max_over_ranks(float(np.mean(bwd_ms)), world)
     # 8 d per unmasked (query, key) pair: the dV, dP, dQ and dK contractions
-    bwd_flops = 2.0 * flops
+    bwd_flops = 2.0 * p32.flops()
     bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    assert ssa.ssa_device_error() == 0
 
-    tc = ssa.ssa_sparse_attn_uses_tensor_cores(Q.dtype, cp.Hq, cp.Hkv, cp.d, cp.B)
-    kernels = {
-        "ssa_block_summary": {"ms": float(seg_mean[0]), "bound": "hbm",
-                              "GB/s": sum_bytes / (seg_mean[0] * 1e-3) / 1e9},
-        "ssa_route": {"ms": float(seg_mean[1]), "bound": "hbm",
-                      "GB/s": route_bytes / (seg_mean[1] * 1e-3) / 1e9},
-        "ssa_sparse_attn_fwd": {"ms": attn_ms, "bound": "tensor" if tc else "alu",
-                                "TFLOP/s": attn_tflops},
-        "ssa_decode": {"ms": float(seg_mean[3]), "bound": "hbm", "GB/s": dec_gbs,
-                       "tokens/s": dec_tok},
-        "ssa_decode_append": {"ms": app_ms, "bound": "hbm",
-                              "GB/s": app_bytes / (app_ms * 1e-3) / 1e9,
-                              "note": "timed apart from the step (CUDA graph of 20 calls); "
-                                      "every append completes a block"},
-        "ssa_sparse_attn_bwd": {"ms": bwd_ms, "bound": "tensor", "TFLOP/s": bwd_tflops,
-                                "frac_bf16": bwd_tflops / bf16_peak,
-                                "work_per_launch": f"{bwd_flops:.4e} FLOP",
-                                "note": "timed apart from the step; FLOPs = 8 d per unmasked "
-                                        "(query, key) pair, the recomputed S not counted"},
-    }
-    for k, v in kernels.items():
-        if "GB/s" in v:
-            v["frac_hbm"] = v["GB/s"] / hbm_peak
-    kernels["ssa_sparse_attn_fwd"]["frac_bf16"] = attn_tflops / bf16_peak
+    kernels = {k: head_rep[k] for k in ("ssa_block_summary", "ssa_route", "ssa_sparse_attn_fwd")}
+    kernels["ssa_decode"] = {"ms": decode_ms, "bound": "hbm", "GB/s": dec_gbs,
+                             "tokens/s": dec_tok, **fracs(dec_gbs, hbm_peak, NOMINAL_HBM_GBS),
+                             "bytes": dbytes}
+    kernels["ssa_decode_append"] = {
+        "ms": app_ms, "bound": "hbm", "GB/s": app_gbs, **fracs(app_gbs, hbm_peak, NOMINAL_HBM_GBS),
+        "note": "timed apart from the step (CUDA graph of 20 calls); every append completes a "
+                "block; launch-bound at 8.9 MB per call"}
+    kernels["ssa_sparse_attn_bwd"] = {
+        "ms": bwd_ms, "bound": "tensor", "TFLOP/s": bwd_tflops,
+        **fracs(bwd_tflops, bf16_peak, NOMINAL_BF16_TFLOPS),
+        "work_per_launch": f"{bwd_flops:.4e} FLOP", "workload": describe(c32),
+        "note": "timed apart from the step; FLOPs = 8 d per unmasked (query, key) pair, the "
+                "recomputed S not counted"}
     roof = {"kernel": "ssa_sparse_attn_fwd", "bound": "tensor" if tc else "alu",
             "achieved": attn_tflops, "peak": bf16_peak, "unit": "TFLOP/s",
-            "frac": attn_tflops / bf16_peak, "traffic": attn_traffic_per_launch(),
+            "frac": attn_tflops / bf16_peak,
+            "traffic": traffic_per_launch(f"attn_tc_{head}_traffic.txt", "attn_tc.cu"),
             "traffic_unit": "bytes per launch (ncu dram read+write, profiles/)",
-            "peak_source": f"{peak_kind} bf16 dense (burst)",
+            "peak_source": f"{peak_kind} bf16 dense (burst), MEASURED_PEAKS.json",
+            "frac_nominal": attn_tflops / NOMINAL_BF16_TFLOPS,
+            "nominal_peak": NOMINAL_BF16_TFLOPS,
             "work_per_launch": f"{flops:.4e} FLOP"}
 
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded planted-cluster Q/K/V; no model weights)",
-        "config": {"workload": "prefill32k (1x32q/8kv, N=32768, d=128, bf16, B=64, top-k=16) "
-                               "+ decode (64 seq x 65536, 32q/8kv, d=128, bf16, B=64, top-k=32)",
-                   "l2": "no flush: inputs larger than L2 (Q 256 MiB; decode reads ~840 MB)",
+        "data": "synthetic (seeded planted-cluster Q/K/V drawn on the device; no model weights)",
+        "config": {"workload": f"{describe(cp)} + decode (64 seq x 65536, 32q/8kv, d=128, bf16, "
+                               f"B=64, top-k=32)",
+                   "l2": "no flush: inputs larger than L2 (Q 1 GiB at 128K, 256 MiB at 32K; "
+                         "decode reads ~840 MB)",
                    "parallelism": f"replicas x{world} (independent problems, no collective)"},
-        "prefill_ms": prefill_ms, "decode": {"tokens_per_s": dec_tok, "ms": decode_ms,
-                                             "GB/s": dec_gbs, "frac_hbm": dec_gbs / hbm_peak,
-                                             "bytes_per_step": dbytes},
+        "prefill_ms": prefill_ms,
+        "decode": {"tokens_per_s": dec_tok, "ms": decode_ms, "GB/s": dec_gbs,
+                   **fracs(dec_gbs, hbm_peak, NOMINAL_HBM_GBS), "bytes_per_step": dbytes},
         "kernels": kernels, "roofline": roof,
+        other: other_rep,
+        "sweep": {"workload": describe(cs, "k"),
+                  "points": sweep},
         "e2e": {"value": all_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * 5,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+        result["cpu_baseline"] = cpu_baseline(head, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(result))
     if world > 1:
@@ -433,18 +569,19 @@ def run_ours(args, world, rank, local):
 
 
 # ------------------------------------------------------------ oracle (CPU) arm
-def _oracle_prefill_sample(nblocks: int, seed: int = 0):
-    """Oracle summary + routing + attention on KV head 0 of the 32K workload,
-    attention restricted to `nblocks` query blocks spread over the sequence."""
+def _oracle_prefill_sample(name: str, nblocks: int, seed: int = 0):
+    """Oracle summary + routing + attention on KV head 0 of a prefill workload
+    (its 4 query heads), attention restricted to `nblocks` query blocks spread
+    over the sequence.  Returns (selected-block FLOPs of the attended blocks,
+    seconds)."""
     import oracle as O
     from workloads import to_f64
-    cp = CONFIGS["prefill32k"]
+    cp = CONFIGS[name]
     G = cp.Hq // cp.Hkv
-    Q, K, V = planted_prefill(cp.batch, cp.Hq, cp.Hkv, cp.N, cp.d, cp.B, cp.clusters,
-                              seed=cp.seed + seed, dtype=cp.dtype)
-    Qf = to_f64(Q[:, :G])
-    Kf = to_f64(K[:, :1])
-    Vf = to_f64(V[:, :1])
+    Q, K, V = planted_prefill(1, G, 1, cp.N, cp.d, cp.B, cp.clusters, seed=cp.seed + seed,
+                              dtype=cp.dtype)
+    Qf, Kf, Vf = to_f64(Q), to_f64(K), to_f64(V)
+    del Q, K, V
     t0 = time.perf_counter()
     S = O.block_summary(Kf, cp.B)
     idx, cnt, _ = O.route(Qf, S, cp.B, cp.topk, 1)
@@ -452,51 +589,73 @@ def _oracle_prefill_sample(nblocks: int, seed: int = 0):
     picks = np.linspace(0, nq - 1, nblocks).astype(int)
     O.sparse_attention(Qf, Kf, Vf, idx, cnt, cp.B, units=[(0, 0, int(i)) for i in picks])
     dt = time.perf_counter() - t0
-    sub = np.zeros_like(cnt[0, 0])
-    sub[picks] = cnt[0, 0, picks]
     rows = np.minimum(cp.B, cp.N - picks * cp.B).astype(np.float64)
     pairs = (rows * cp.B * (cnt[0, 0, picks] - 1) + rows * (rows + 1) / 2).sum()
-    flops = pairs * G * 4 * cp.d
-    return flops, dt
+    return pairs * G * 4 * cp.d, dt
 
 
-def cpu_baseline(budget_s: float = 15.0):
+def _oracle_decode_sample(nseq: int, seed: int = 0):
+    """Oracle decode step (fp64 summaries of the cache, routing, attention) on
+    `nseq` sequences of the decode workload.  Returns (tokens, seconds)."""
+    import oracle as O
+    from workloads import to_f64
+    cd = CONFIGS["decode"]
+    q, Kc, Vc, L = planted_decode(nseq, cd.Hq, cd.Hkv, cd.L, cd.d, cd.B, cd.clusters,
+                                  seed=cd.seed + seed, dtype=cd.dtype)
+    qf, Ls = to_f64(q), L.numpy()
+    Kc, Vc = Kc.float().numpy(), Vc.float().numpy()  # exact; widened to fp64 by the oracle
+    t0 = time.perf_counter()
+    S = np.stack([O.block_summary(Kc[b:b + 1], cd.B)[0] for b in range(nseq)])
+    O.decode(qf, Kc, Vc, Ls, cd.B, cd.topk, S=S)
+    return nseq, time.perf_counter() - t0
+
+
+def cpu_baseline(name: str, budget_s: float = 15.0):
     cores = len(os.sched_getaffinity(0))
     # calibrate the number of attended query blocks to fit the budget
-    f, dt = _oracle_prefill_sample(8)
-    n = int(max(8, min(512, 8 * budget_s / max(dt, 1e-3))))
-    f, dt = _oracle_prefill_sample(n)
+    f, dt = _oracle_prefill_sample(name, 4)
+    n = int(max(4, min(CONFIGS[name].N // CONFIGS[name].B, 4 * budget_s / max(dt, 1e-3))))
+    f, dt = _oracle_prefill_sample(name, n)
+    tok, ddt = _oracle_decode_sample(2)
+    nq = CONFIGS[name].N // CONFIGS[name].B
     return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"fp64 numpy oracle on the 32K prefill workload, KV head 0 (4 query heads): "
-                      f"summary + routing of all 512 query blocks, attention of {n} query blocks "
+            "sample": f"fp64 numpy oracle on the {name} workload, KV head 0 (its 4 query heads): "
+                      f"summary + routing of all {nq} query blocks, attention of {n} query blocks "
                       f"spread over the sequence; {dt:.1f} s; FLOPs = selected-block FLOPs of "
                       f"the attended blocks",
-            "threads": torch.get_num_threads()}
+            "threads": torch.get_num_threads(),
+            "decode": {"tokens_per_s": tok / ddt, "seconds": ddt,
+                       "sample": f"{tok} of the 64 decode sequences: fp64 summaries of the "
+                                 f"65536-token cache, routing and attention"}}
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return
+    name = args.workload
     cores = len(os.sched_getaffinity(0))
     for _ in range(args.warmup):
-        _oracle_prefill_sample(4)
+        _oracle_prefill_sample(name, 2)
     times, flops = [], 0.0
     for k in range(args.steps):
-        f, dt = _oracle_prefill_sample(16, seed=k)
+        f, dt = _oracle_prefill_sample(name, 4, seed=k)
         times.append(dt)
         flops = f
+    tok, ddt = _oracle_decode_sample(1)
     ms = float(np.mean(times)) * 1e3
     value = flops / (ms * 1e-3) / 1e12
+    c = CONFIGS[name]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded planted-cluster Q/K/V; no model weights)",
-        "config": {"workload": "prefill32k (1x32q/8kv, N=32768, d=128, bf16, B=64, top-k=16); "
-                               "CPU sample: KV head 0, 16 attended query blocks per step"},
+        "config": {"workload": f"{describe(c)}; CPU sample: KV head 0, summary + routing of "
+                               f"every query block and attention of 4 query blocks per step"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": "fp64 oracle: summary + routing of KV head 0, attention of "
-                                   "16 query blocks per step"},
+                         "sample": f"fp64 oracle: summary + routing of KV head 0 of {name}, "
+                                   f"attention of 4 query blocks per step",
+                         "decode_tokens_per_s": tok / ddt},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -506,8 +665,8 @@ def run_reference(args, world, rank):
 def run_ncu_case(case: str, launches: int):
     """Run one kernel of the hot path `launches` times on a bounded workload
     (a few GB on the device, working set above the 126 MB L2) for profiling:
-    summary / route / attn on the 32K prefill workload, decode on 16 of the 64
-    sequences of the decode workload."""
+    summary / route / attn / bwd on the 32K prefill workload, attn128k on the
+    128K one, decode on 16 of the 64 sequences of the decode workload."""
     import block_sparse_top_summary_b200 as ssa
     ssa.load_library()
     dev = torch.device("cuda", 0)
@@ -520,20 +679,21 @@ def run_ncu_case(case: str, launches: int):
         for _ in range(launches):
             ssa.ssa_decode(q, Kc, Vc, Sc, L, cd.B, cd.topk)
     else:
-        cp = CONFIGS["prefill32k"]
-        Q, K, V = planted_prefill(cp.batch, cp.Hq, cp.Hkv, cp.N, cp.d, cp.B, cp.clusters,
-                                  seed=cp.seed, dtype=cp.dtype)
-        Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
-        S = ssa.ssa_block_summary(Kd, cp.B)
-        idx, cnt = ssa.ssa_route(Qd, S, cp.B, cp.topk, cp.Hkv)
+        cp = CONFIGS["prefill128k" if case.endswith("128k") else "prefill32k"]
+        p = Prefill(ssa, cp, dev, cp.seed)
+        p.run()
         torch.cuda.synchronize()
+        if case == "bwd":
+            dO = upstream_grad(cp.batch, cp.Hq, cp.N, cp.d, seed=1, dtype=cp.dtype, device=dev)
         for _ in range(launches):
             if case == "summary":
-                ssa.ssa_block_summary(Kd, cp.B, S=S)
-            elif case == "route":
-                ssa.ssa_route(Qd, S, cp.B, cp.topk, cp.Hkv, idx=idx, cnt=cnt)
+                ssa.ssa_block_summary(p.K, cp.B, S=p.S)
+            elif case.startswith("route"):
+                ssa.ssa_route(p.Q, p.S, cp.B, cp.topk, cp.Hkv, idx=p.idx, cnt=p.cnt)
+            elif case == "bwd":
+                ssa.ssa_sparse_attn_bwd(p.Q, p.K, p.V, p.O, dO, p.lse, p.idx, p.cnt, cp.B)
             else:
-                ssa.ssa_sparse_attn_fwd(Qd, Kd, Vd, idx, cnt, cp.B)
+                ssa.ssa_sparse_attn_fwd(p.Q, p.K, p.V, p.idx, p.cnt, cp.B, O=p.O, lse=p.lse)
     torch.cuda.synchronize()
     assert ssa.ssa_device_error() == 0
     print(f"ncu case {case}: {launches} launches done")
@@ -542,12 +702,16 @@ def run_ncu_case(case: str, launches: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill128k", "prefill32k"], default="prefill128k",
+                    help="the prefill workload of the timed step")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["summary", "route", "attn", "decode"], default=None,
+    ap.add_argument("--ncu-case", default=None,
+                    choices=["summary", "route", "attn", "bwd", "decode", "route128k",
+                             "attn128k"],
                     help="run one kernel on a bounded workload for profiling, then exit")
     ap.add_argument("--ncu-launches", type=int, default=2)
     args = ap.parse_args()

@@ -12,6 +12,7 @@ from .abi import (  # noqa: F401
     prefill,
     route_width,
     ssa_block_summary,
+    ssa_check_device_error,
     ssa_decode,
     ssa_decode_append,
     ssa_decode_noalloc,

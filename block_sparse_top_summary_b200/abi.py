@@ -22,10 +22,11 @@ SSA_BF16 = 1
 _STATUS = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED", 3: "SSA_ERR_CUDA",
            4: "SSA_ERR_TIMEOUT"}
 
-# Every symbol include/ssa.h declares.
+# Every symbol include/ssa.h and include/ssa_debug.h declare.
 EXPORTS = ("ssa_status_string", "ssa_version", "ssa_block_summary", "ssa_route",
-           "ssa_sparse_attn_fwd", "ssa_sparse_attn_uses_tensor_cores", "ssa_decode_workspace_size",
-           "ssa_decode", "ssa_device_error", "ssa_sparse_attn_bwd")
+           "ssa_sparse_attn_fwd", "ssa_sparse_attn_bwd", "ssa_sparse_attn_uses_tensor_cores",
+           "ssa_decode_workspace_size", "ssa_decode", "ssa_decode_append", "ssa_decode_noalloc",
+           "ssa_device_error", "ssa_check_device_error", "ssa_debug_wait_timeout")
 
 
 class SSAError(RuntimeError):
@@ -53,11 +54,17 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.ssa_status_string.argtypes = [i]
     lib.ssa_version.restype = i
     lib.ssa_block_summary.argtypes = [vp, i, i, i, i, i, i, vp, vp]
-    lib.ssa_route.argtypes = [vp, i, vp, i, i, i, i, i, i, i, i, vp, vp, vp]
+    lib.ssa_route.argtypes = [vp, i, vp, i, i, i, i, i, i, i, i, vp, vp, vp, vp]
     lib.ssa_sparse_attn_fwd.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp]
     lib.ssa_decode_workspace_size.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(sz)]
     lib.ssa_decode.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, sz, vp]
     lib.ssa_device_error.argtypes = [ctypes.POINTER(i)]
+    lib.ssa_check_device_error.argtypes = [vp, ctypes.POINTER(i)]
+    lib.ssa_decode_noalloc.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp]
+    lib.ssa_decode_append.argtypes = [vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.ssa_sparse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f,
+                                        vp, vp, vp, vp, vp]
+    lib.ssa_debug_wait_timeout.argtypes = [i, vp]
     lib.ssa_sparse_attn_uses_tensor_cores.argtypes = [i, i, i, i, i]
     for name in EXPORTS:
         if name not in ("ssa_status_string", "ssa_version"):
@@ -114,8 +121,11 @@ def route_width(N: int, B: int, topk: int) -> int:
 
 
 def ssa_route(Q: torch.Tensor, S: torch.Tensor, B: int, topk: int, Hkv: int,
-              max_sel: int | None = None, idx=None, cnt=None, stream=None):
-    """Top-k routing per (batch, KV head, query block): returns ``(idx, cnt)``."""
+              max_sel: int | None = None, idx=None, cnt=None, scores=None,
+              want_scores: bool = False, stream=None):
+    """Top-k routing per (batch, KV head, query block): returns ``(idx, cnt)``,
+    or ``(idx, cnt, scores)`` when ``scores`` is given or ``want_scores`` is set
+    (``scores``: ``[batch, Hkv, nq, N // B]`` fp32, -inf off the candidates)."""
     _need(Q, "Q")
     batch, Hq, N, d = Q.shape
     nq = -(-N // B)
@@ -125,10 +135,15 @@ def ssa_route(Q: torch.Tensor, S: torch.Tensor, B: int, topk: int, Hkv: int,
         idx = torch.empty(batch, Hkv, nq, max_sel, dtype=torch.int32, device=Q.device)
     if cnt is None:
         cnt = torch.empty(batch, Hkv, nq, dtype=torch.int32, device=Q.device)
+    ret_scores = scores is not None or want_scores
+    if scores is None and want_scores:
+        scores = torch.empty(batch, Hkv, nq, N // B, dtype=torch.float32, device=Q.device)
+    if scores is not None:
+        _need(scores, "scores")
     _check("ssa_route", load_library().ssa_route(
         _ptr(Q), _dtype_code(Q), _ptr(S), batch, Hq, Hkv, N, d, B, topk, max_sel, _ptr(idx),
-        _ptr(cnt), _stream(stream)))
-    return idx, cnt
+        _ptr(cnt), _ptr(scores), _stream(stream)))
+    return (idx, cnt, scores) if ret_scores else (idx, cnt)
 
 
 def ssa_sparse_attn_fwd(Q, K, V, idx, cnt, B: int, scale: float | None = None, O=None, lse=None,
@@ -199,6 +214,15 @@ def ssa_device_error() -> int:
     return code.value
 
 
+def ssa_check_device_error(stream=None) -> int:
+    """Read and reset the device-side error word in the order of ``stream``,
+    waiting for that stream only."""
+    code = ctypes.c_int(0)
+    _check("ssa_check_device_error", load_library().ssa_check_device_error(
+        _stream(stream), ctypes.byref(code)))
+    return code.value
+
+
 def prefill(Q, K, V, B: int, topk: int, scale: float | None = None, stream=None):
     """The three prefill calls in order: summary, route, attention.
 
@@ -219,11 +243,7 @@ def ssa_decode_noalloc(q, Kc, Vc, S, seqlens, B: int, topk: int, scale: float | 
     """
     for t, n in ((q, "q"), (Kc, "Kc"), (Vc, "Vc"), (seqlens, "seqlens")):
         _need(t, n)
-    lib = load_library()
-    fn = lib.ssa_decode_noalloc
-    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    fn.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp]
-    fn.restype = i
+    fn = load_library().ssa_decode_noalloc
     batch, Hq, d = q.shape
     Hkv, Lmax = Kc.shape[1], Kc.shape[2]
     if scale is None:
@@ -249,11 +269,7 @@ def ssa_decode_append(Kc, Vc, S, seqlens, k_new, v_new, B: int, stream=None):
     for t, n in ((Kc, "Kc"), (Vc, "Vc"), (S, "S"), (seqlens, "seqlens"), (k_new, "k_new"),
                  (v_new, "v_new")):
         _need(t, n)
-    lib = load_library()
-    fn = lib.ssa_decode_append
-    vp, i = ctypes.c_void_p, ctypes.c_int
-    fn.argtypes = [vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, vp]
-    fn.restype = i
+    fn = load_library().ssa_decode_append
     batch, Hkv, Lmax, d = Kc.shape
     _check("ssa_decode_append", fn(
         _ptr(Kc), _ptr(Vc), _dtype_code(Kc), _ptr(S), _ptr(seqlens), _ptr(k_new), _ptr(v_new),
@@ -272,11 +288,7 @@ def ssa_sparse_attn_bwd(Q, K, V, O, dO, lse, idx, cnt, B: int, scale: float | No
     for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O"), (dO, "dO"), (lse, "lse"), (idx, "idx"),
                  (cnt, "cnt")):
         _need(t, n)
-    lib = load_library()
-    fn = lib.ssa_sparse_attn_bwd
-    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    fn.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, vp, vp]
-    fn.restype = i
+    fn = load_library().ssa_sparse_attn_bwd
     batch, Hq, N, d = Q.shape
     Hkv = K.shape[1]
     if scale is None:
@@ -298,6 +310,4 @@ def ssa_debug_wait_timeout(limit_us: int, stream=None):
     """Run the bounded-wait self-test (include/ssa_debug.h); read the result with
     ssa_device_error()."""
     fn = load_library().ssa_debug_wait_timeout
-    fn.argtypes = [ctypes.c_int, ctypes.c_void_p]
-    fn.restype = ctypes.c_int
     _check("ssa_debug_wait_timeout", fn(limit_us, _stream(stream)))

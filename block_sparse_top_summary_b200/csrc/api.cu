@@ -21,6 +21,26 @@ ssa_status check_dims(int d, int B, ssa_dtype dt) {
 
 ssa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA; }
 
+// Result word of ssa_check_device_error (one per device).
+__device__ int g_error_taken = 0;
+
+constexpr int kMaxErrorWords = 4;
+struct ErrorWords {
+  int* w[kMaxErrorWords];
+  int n;
+};
+
+// Takes every error word (atomic exchange with 0) and stores the first
+// non-zero one, in the order given, into g_error_taken.
+__global__ void take_error_words_kernel(ErrorWords words) {
+  int first = 0;
+  for (int k = 0; k < words.n; ++k) {
+    const int v = atomicExch(words.w[k], 0);
+    if (first == 0) first = v;
+  }
+  g_error_taken = first;
+}
+
 }  // namespace
 
 extern "C" {
@@ -36,7 +56,7 @@ const char* ssa_status_string(int status) {
   }
 }
 
-int ssa_version(void) { return 102; }
+int ssa_version(void) { return 200; }
 
 ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv, int N, int d,
                              int B, float* S, ssa_stream stream) {
@@ -52,7 +72,7 @@ ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv,
 
 ssa_status ssa_route(const void* Q, ssa_dtype dtype, const float* S, int batch, int Hq, int Hkv,
                      int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
-                     ssa_stream stream) {
+                     float* scores, ssa_stream stream) {
   ssa_status st = check_dims(d, B, dtype);
   if (st != SSA_OK) return st;
   if (batch <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || topk < 0) return SSA_ERR_INVALID_ARG;
@@ -65,8 +85,9 @@ ssa_status ssa_route(const void* Q, ssa_dtype dtype, const float* S, int batch, 
   if (Q == nullptr || idx == nullptr || cnt == nullptr) return SSA_ERR_INVALID_ARG;
   if (N / B > 0 && S == nullptr) return SSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(S)) return SSA_ERR_INVALID_ARG;
+  if (scores != nullptr && !aligned16(scores)) return SSA_ERR_INVALID_ARG;
   return from_cuda(ssa::launch_route(Q, dtype, S, batch, Hq, Hkv, N, d, B, topk, max_sel, idx, cnt,
-                                     reinterpret_cast<cudaStream_t>(stream)));
+                                     scores, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 ssa_status ssa_sparse_attn_fwd(const void* Q, const void* K, const void* V, ssa_dtype dtype,
@@ -180,6 +201,24 @@ ssa_status ssa_device_error(int* code) {
   int a = ssa::read_and_reset_attn_tc_error();
   int b = ssa::read_and_reset_decode_error();
   *code = a != 0 ? a : b;
+  return SSA_OK;
+}
+
+ssa_status ssa_check_device_error(ssa_stream stream, int* code) {
+  if (code == nullptr) return SSA_ERR_INVALID_ARG;
+  ErrorWords words{};
+  if (ssa::attn_tc_error_word(&words.w[0]) != cudaSuccess) return SSA_ERR_CUDA;
+  if (ssa::decode_error_word(&words.w[1]) != cudaSuccess) return SSA_ERR_CUDA;
+  words.n = 2;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  take_error_words_kernel<<<1, 1, 0, s>>>(words);
+  if (cudaGetLastError() != cudaSuccess) return SSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_error_taken, sizeof(int), 0, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return SSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SSA_ERR_CUDA;
+  *code = v;
   return SSA_OK;
 }
 

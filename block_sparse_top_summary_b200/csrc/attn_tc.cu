@@ -705,6 +705,10 @@ cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const in
                                     st);
 }
 
+cudaError_t attn_tc_error_word(int** word) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(word), g_attn_tc_error);
+}
+
 int read_and_reset_attn_tc_error() {
   int v = 0;
   cudaMemcpyFromSymbol(&v, g_attn_tc_error, sizeof(int));

@@ -1300,6 +1300,10 @@ cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, co
                                                scale, O, idx_out, ws, st);
 }
 
+cudaError_t decode_error_word(int** word) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(word), g_decode_error);
+}
+
 int read_and_reset_decode_error() {
   int v = 0;
   cudaMemcpyFromSymbol(&v, g_decode_error, sizeof(int));

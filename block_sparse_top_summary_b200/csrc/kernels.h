@@ -18,7 +18,7 @@ constexpr int kRouteMaxBlocks = 4096;
 
 cudaError_t launch_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq, int Hkv,
                          int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
-                         cudaStream_t st);
+                         float* scores, cudaStream_t st);
 
 // True when the tensor-core prefill kernel covers this shape.
 bool attn_tc_supported(ssa_dtype dt, int Hq, int Hkv, int d, int B);
@@ -65,5 +65,8 @@ cudaError_t launch_decode_append(void* Kc, void* Vc, ssa_dtype dt, float* S, int
 // read and reset; returns the first non-zero code or 0.
 int read_and_reset_attn_tc_error();
 int read_and_reset_decode_error();
+// Device addresses of the same words (current device), for stream-ordered reads.
+cudaError_t attn_tc_error_word(int** word);
+cudaError_t decode_error_word(int** word);
 
 }  // namespace ssa

@@ -18,7 +18,8 @@
 //      product l in lane l; scores land in shared memory;
 //   3. select: warp w selects for query block w of the tile with an exact
 //      4-pass radix select (ties to the lower index) and writes the ascending
-//      block list.
+//      block list, and, when the caller asks for them, the block's row of
+//      scores (-inf where a block is not a candidate).
 // Tiles are dispatched heaviest first (late query blocks have the most
 // candidates).
 #include "common.cuh"
@@ -53,7 +54,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
                                                     const float* __restrict__ S,
                                                     int32_t* __restrict__ idx,
-                                                    int32_t* __restrict__ cnt, int Hq, int Hkv,
+                                                    int32_t* __restrict__ cnt,
+                                                    float* __restrict__ scores, int Hq, int Hkv,
                                                     int N, int B, int nq, int nfull, int topk,
                                                     int max_sel, int ntiles, int sc_stride,
                                                     float inv_sqrt_d) {
@@ -188,6 +190,12 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
         cnt[(int64_t)bg * nq + i] = n_sel;
       }
       for (int p = n_sel + lane; p < max_sel; p += 32) row[p] = -1;
+      if (scores != nullptr) {
+        float* srow = scores + ((int64_t)bg * nq + i) * nfull;
+        const float* mine = sc + warp * sc_stride;
+        for (int j = lane; j < nfull; j += 32)
+          srow[j] = (j >= 1 && j <= i - 1) ? mine[j - 1] : -INFINITY;
+      }
     }
   }
 }
@@ -195,7 +203,7 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
 template <typename T, int D>
 static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int Hq, int Hkv, int N,
                                   int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
-                                  cudaStream_t st) {
+                                  float* scores, cudaStream_t st) {
   const int nq = (N + B - 1) / B;
   const int nfull = N / B;
   const int ntiles = (nq + TQ - 1) / TQ;
@@ -205,7 +213,8 @@ static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(batch * Hkv, ntiles);
-  route_kernel<T, D><<<grid, 256, smem, st>>>((const T*)Q, S, idx, cnt, Hq, Hkv, N, B, nq, nfull,
+  route_kernel<T, D><<<grid, 256, smem, st>>>((const T*)Q, S, idx, cnt, scores, Hq, Hkv, N, B,
+                                              nq, nfull,
                                               topk, max_sel, ntiles, sc_stride,
                                               1.0f / sqrtf((float)D));
   return cudaGetLastError();
@@ -213,17 +222,17 @@ static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int 
 
 cudaError_t launch_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq, int Hkv,
                          int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
-                         cudaStream_t st) {
+                         float* scores, cudaStream_t st) {
   if (dt == SSA_BF16) {
     return d == 128 ? launch_route_t<__nv_bfloat16, 128>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel,
-                                                         idx, cnt, st)
+                                                         idx, cnt, scores, st)
                     : launch_route_t<__nv_bfloat16, 64>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel,
-                                                        idx, cnt, st);
+                                                        idx, cnt, scores, st);
   }
   return d == 128 ? launch_route_t<float, 128>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt,
-                                               st)
+                                               scores, st)
                   : launch_route_t<float, 64>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt,
-                                              st);
+                                              scores, st);
 }
 
 }  // namespace ssa

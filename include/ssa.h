@@ -56,7 +56,8 @@ typedef struct CUstream_st* ssa_stream;
 const char* ssa_status_string(int status);
 
 /* Library ABI version (major * 100 + minor).  1.01 added ssa_decode_append,
- * 1.02 ssa_sparse_attn_bwd. */
+ * 1.02 ssa_sparse_attn_bwd; 2.00 added the `scores` output of ssa_route (an
+ * incompatible signature change) and ssa_check_device_error. */
 int ssa_version(void);
 
 /*
@@ -89,6 +90,10 @@ ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv,
  * Q: [batch, Hq, N, d] of `dtype`.  S: [batch, Hkv, nfull, d] fp32.
  * idx: [batch, Hkv, nq, max_sel] int32 (written; entries past cnt are -1).
  * cnt: [batch, Hkv, nq] int32 (written).
+ * scores: NULL, or [batch, Hkv, nq, nfull] fp32 (written): scores[b, g, i, j]
+ *    is the fp32 score s_j that the selection ranked, for the candidates
+ *    j = 1 .. i-1, and -inf for every other j (the sink, the diagonal block
+ *    and later blocks).  16-byte aligned.
  * topk >= 0; any topk >= nq selects every candidate.
  * max_sel must be >= min(topk, max(nq - 2, 0)) + 2.
  * SSA_ERR_UNSUPPORTED if nq > 4096 (the score rows of a tile of query blocks
@@ -96,7 +101,7 @@ ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv,
  */
 ssa_status ssa_route(const void* Q, ssa_dtype dtype, const float* S, int batch, int Hq, int Hkv,
                      int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
-                     ssa_stream stream);
+                     float* scores, ssa_stream stream);
 
 /*
  * Stage 2, exact softmax attention over the selected blocks (SSA page,
@@ -264,6 +269,18 @@ ssa_status ssa_decode_noalloc(const void* q, const void* Kc, const void* Vc, ssa
  * writes the word to *code and resets it to 0.
  */
 ssa_status ssa_device_error(int* code);
+
+/*
+ * The device error word, read in stream order: enqueues on `stream` a
+ * one-thread kernel that takes the word (atomic exchange with 0), copies it
+ * back, and waits for `stream` only (cudaStreamSynchronize; other streams
+ * keep running).  *code is 0, or the ssa_status of the first bounded wait that
+ * expired in work that finished before that kernel ran, on any stream of the
+ * current device.  The copy goes through one result word of the library per
+ * device: calls from several host threads at once must be serialised.  Not
+ * for use during stream capture (it synchronises).
+ */
+ssa_status ssa_check_device_error(ssa_stream stream, int* code);
 
 #ifdef __cplusplus
 }

@@ -35,14 +35,14 @@ def test_every_declared_symbol_is_exported(lib):
     assert "ssa_route" in declared and "ssa_decode" in declared
     for name in declared:
         assert hasattr(lib, name), name
-    assert set(abi.EXPORTS) <= set(declared)
+    assert set(abi.EXPORTS) == set(declared)
 
 
 def test_status_strings_and_version(lib):
     assert lib.ssa_status_string(0) == b"SSA_OK"
     assert lib.ssa_status_string(4) == b"SSA_ERR_TIMEOUT"
     assert lib.ssa_status_string(99) == b"SSA_ERR_UNKNOWN"
-    assert lib.ssa_version() >= 102
+    assert lib.ssa_version() >= 200
 
 
 NULL = None
@@ -59,18 +59,24 @@ def test_summary_rejects_bad_arguments(lib):
 
 
 def test_route_rejects_bad_arguments(lib):
-    args = dict(Q=FAKE, dt=1, S=FAKE, b=1, Hq=4, Hkv=2, N=1024, d=128, B=64, k=4, w=6)
+    args = dict(Q=FAKE, dt=1, S=FAKE, b=1, Hq=4, Hkv=2, N=1024, d=128, B=64, k=4, w=6,
+                scores=NULL)
 
     def call(**kw):
         a = {**args, **kw}
         return lib.ssa_route(a["Q"], a["dt"], a["S"], a["b"], a["Hq"], a["Hkv"], a["N"], a["d"],
-                             a["B"], a["k"], a["w"], FAKE, FAKE, NULL)
+                             a["B"], a["k"], a["w"], FAKE, FAKE, a["scores"], NULL)
 
     assert call(Hq=5) == 1           # Hq % Hkv
     assert call(k=-1) == 1           # negative top-k
     assert call(w=5) == 1            # idx row too narrow for k + 2
     assert call(Q=NULL) == 1
     assert call(N=64 * 5000) == 2    # more query blocks than the kernel holds
+    assert call(scores=ctypes.c_void_p(0x100004)) == 1  # scores not 16-byte aligned
+
+
+def test_check_device_error_needs_an_output(lib):
+    assert lib.ssa_check_device_error(NULL, NULL) == 1
 
 
 def test_attn_rejects_bad_arguments(lib):
@@ -105,9 +111,6 @@ def test_decode_workspace_and_rejections(lib):
 
 def test_decode_append_rejections(lib):
     fn = lib.ssa_decode_append
-    vp, i = ctypes.c_void_p, ctypes.c_int
-    fn.argtypes = [vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, vp]
-    fn.restype = i
     ok = (FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 4, 2, 1024, 128, 64, NULL)
 
     def call(**kw):
@@ -130,9 +133,6 @@ def test_decode_append_rejections(lib):
 
 def test_attention_backward_rejections(lib):
     fn = lib.ssa_sparse_attn_bwd
-    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    fn.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp, vp, vp]
-    fn.restype = i
     names = ["Q", "K", "V", "O", "dO", "lse", "dt", "idx", "cnt", "batch", "Hq", "Hkv", "N", "d",
              "B", "max_sel", "scale", "dQ", "dK", "dV", "delta", "stream"]
     ok = [FAKE] * 6 + [1, FAKE, FAKE, 1, 8, 2, 4096, 128, 64, 18, 0.088, FAKE, FAKE, FAKE, FAKE,

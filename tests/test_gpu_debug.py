@@ -27,3 +27,16 @@ def test_bounded_wait_expires_and_context_survives():
     ma, _ = out_errors(to_f64(out), ref)
     assert ma <= BF16_MAX_ABS
     assert ssa.ssa_device_error() == 0
+
+
+def test_stream_ordered_error_check():
+    # The same expired wait, read back in the order of the stream it ran on,
+    # waiting for that stream only.
+    import block_sparse_top_summary_b200 as ssa
+    assert ssa.ssa_device_error() == 0
+    side = torch.cuda.Stream()
+    ssa.ssa_debug_wait_timeout(2000, stream=side)
+    assert ssa.ssa_check_device_error(side) == 4  # SSA_ERR_TIMEOUT, then reset
+    assert ssa.ssa_check_device_error(side) == 0
+    assert ssa.ssa_check_device_error() == 0  # the current stream
+    assert ssa.ssa_device_error() == 0

@@ -90,6 +90,42 @@ def test_route_parity(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters):
     assert near <= max(1, rows // 50)
 
 
+@pytest.mark.parametrize("batch,Hq,Hkv,N,d,B,topk,dtype", [
+    (1, 8, 2, 64 * 70 + 9, 128, 64, 6, "bf16"),   # ragged tail, 9 tiles of 8
+    (2, 4, 4, 32 * 40, 64, 32, 5, "f32"),
+])
+def test_route_scores_output(ssa, batch, Hq, Hkv, N, d, B, topk, dtype):
+    # The optional scores output holds, for every (query block i, block j),
+    # the fp32 score the selection ranked: within fp32 rounding of the
+    # oracle's fp64 q-bar . S_j / sqrt(d) on the candidates 1 .. i-1, -inf
+    # elsewhere.  The GPU's own selection is exactly the top-k of these
+    # scores (ties to the lower index), and passing the output changes
+    # neither idx nor cnt.
+    Q, K, _ = planted_prefill(batch, Hq, Hkv, N, d, B, 4, seed=7, dtype=dtype)
+    Qd = Q.to(DEV)
+    S = ssa.ssa_block_summary(K.to(DEV), B)
+    idx0, cnt0 = ssa.ssa_route(Qd, S, B, topk, Hkv)
+    idx, cnt, sc = ssa.ssa_route(Qd, S, B, topk, Hkv, want_scores=True)
+    assert torch.equal(idx, idx0) and torch.equal(cnt, cnt0)
+    sc = sc.cpu().double().numpy()
+    nq, nfull = -(-N // B), N // B
+    assert sc.shape == (batch, Hkv, nq, nfull)
+    ref = O.summary_scores(O.pool_query_blocks(to_f64(Q), B, Hkv), O.block_summary(to_f64(K), B))
+    i_ = np.arange(nq)[:, None]
+    j_ = np.arange(nfull)[None, :]
+    cand = (j_ >= 1) & (j_ <= i_ - 1)
+    assert np.all(np.isneginf(sc[..., ~cand]))
+    assert np.max(np.abs(sc[..., cand] - ref[..., cand])) <= 1e-5
+    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(batch):
+        for g in range(Hkv):
+            for i in range(nq):
+                c = np.arange(1, max(i, 1))
+                order = np.lexsort((c, -sc[b, g, i, c]))  # score desc, then index asc
+                want = sorted({0, i} | set(c[order[:topk]].tolist()))
+                assert gi[b, g, i, :gc[b, g, i]].tolist() == want, (b, g, i)
+
+
 def test_route_tiny_matches_golden(ssa):
     import json
     import os
