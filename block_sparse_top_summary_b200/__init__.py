@@ -16,8 +16,17 @@ from .abi import (  # noqa: F401
     ssa_decode,
     ssa_decode_append,
     ssa_decode_noalloc,
+    ssa_decode_paged,
+    ssa_decode_append_paged,
     ssa_decode_workspace_size,
     ssa_device_error,
+    entmax_width,
+    ssa_learned_summary,
+    ssa_route_entmax,
+    ssa_route_hierarchical,
+    ssa_decode_per_head,
+    ssa_decode_per_head_workspace_size,
+    ssa_sparse_attn_fwd_prior,
     ssa_route,
     ssa_sparse_attn_bwd,
     ssa_sparse_attn_fwd,

@@ -26,6 +26,9 @@ _STATUS = {0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_UNSUPPORTED", 3: "
 EXPORTS = ("ssa_status_string", "ssa_version", "ssa_block_summary", "ssa_route",
            "ssa_sparse_attn_fwd", "ssa_sparse_attn_bwd", "ssa_sparse_attn_uses_tensor_cores",
            "ssa_decode_workspace_size", "ssa_decode", "ssa_decode_append", "ssa_decode_noalloc",
+           "ssa_decode_paged", "ssa_decode_append_paged", "ssa_learned_summary",
+           "ssa_route_entmax", "ssa_sparse_attn_fwd_prior", "ssa_route_hierarchical",
+           "ssa_decode_per_head", "ssa_decode_per_head_workspace_size",
            "ssa_device_error", "ssa_check_device_error", "ssa_debug_wait_timeout")
 
 
@@ -65,6 +68,17 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.ssa_sparse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f,
                                         vp, vp, vp, vp, vp]
     lib.ssa_debug_wait_timeout.argtypes = [i, vp]
+    lib.ssa_decode_paged.argtypes = [vp, vp, vp, i, vp, vp, i, i, vp, i, i, i, i, i, i, f, vp, vp,
+                                     vp, sz, vp]
+    lib.ssa_decode_append_paged.argtypes = [vp, vp, i, vp, vp, i, i, vp, vp, vp, i, i, i, i, vp]
+    lib.ssa_learned_summary.argtypes = [vp, i, vp, i, i, i, i, i, vp, vp]
+    lib.ssa_route_hierarchical.argtypes = [vp, i, vp, i, i, i, i, i, i, i, i, i, i, vp, vp, vp]
+    lib.ssa_decode_per_head_workspace_size.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(sz)]
+    lib.ssa_decode_per_head.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp,
+                                        sz, vp]
+    lib.ssa_route_entmax.argtypes = [vp, i, vp, i, i, i, i, i, i, f, f, f, i, vp, vp, vp, vp, vp]
+    lib.ssa_sparse_attn_fwd_prior.argtypes = [vp, vp, vp, i, vp, vp, vp, i, i, i, i, i, i, i, f,
+                                              vp, vp, vp]
     lib.ssa_sparse_attn_uses_tensor_cores.argtypes = [i, i, i, i, i]
     for name in EXPORTS:
         if name not in ("ssa_status_string", "ssa_version"):
@@ -275,6 +289,164 @@ def ssa_decode_append(Kc, Vc, S, seqlens, k_new, v_new, B: int, stream=None):
         _ptr(Kc), _ptr(Vc), _dtype_code(Kc), _ptr(S), _ptr(seqlens), _ptr(k_new), _ptr(v_new),
         batch, Hkv, Lmax, d, B, _stream(stream)))
     return Kc, Vc, S, seqlens
+
+
+def ssa_decode_paged(q, Kp, Vp, S, page_table, seqlens, B: int, topk: int,
+                     scale: float | None = None, O=None, idx=None, want_idx: bool = True,
+                     workspace=None, stream=None):
+    """One decode step over a paged cache: returns ``(O, idx)``.
+
+    ``Kp``/``Vp``: page pools ``[num_pages, Hkv, B, d]``; ``page_table``:
+    ``[batch, max_blocks]`` int32 (-1: no page); ``S``: ``[batch, Hkv,
+    max_blocks, d]`` fp32 summaries in logical block order.
+    """
+    for t, n in ((q, "q"), (Kp, "Kp"), (Vp, "Vp"), (S, "S"), (page_table, "page_table"),
+                 (seqlens, "seqlens")):
+        _need(t, n)
+    batch, Hq, d = q.shape
+    num_pages, Hkv = Kp.shape[0], Kp.shape[1]
+    max_blocks = page_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(q)
+    if idx is None and want_idx:
+        idx = torch.empty(batch, Hkv, decode_width(max_blocks * B, B, topk), dtype=torch.int32,
+                          device=q.device)
+    nbytes = ssa_decode_workspace_size(batch, Hq, Hkv, max_blocks * B, d, B, topk)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check("ssa_decode_paged", load_library().ssa_decode_paged(
+        _ptr(q), _ptr(Kp), _ptr(Vp), _dtype_code(q), _ptr(S), _ptr(page_table), max_blocks,
+        num_pages, _ptr(seqlens), batch, Hq, Hkv, d, B, topk, ctypes.c_float(scale), _ptr(O),
+        _ptr(idx), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return O, idx
+
+
+def ssa_decode_append_paged(Kp, Vp, S, page_table, seqlens, k_new, v_new, B: int, stream=None):
+    """Append one token per sequence to a paged cache, in place (the row goes
+    to row ``L % B`` of page ``page_table[b, L // B]``; a sequence whose next
+    block has no page is left unchanged)."""
+    for t, n in ((Kp, "Kp"), (Vp, "Vp"), (S, "S"), (page_table, "page_table"),
+                 (seqlens, "seqlens"), (k_new, "k_new"), (v_new, "v_new")):
+        _need(t, n)
+    num_pages, Hkv, _, d = Kp.shape
+    batch, max_blocks = page_table.shape
+    _check("ssa_decode_append_paged", load_library().ssa_decode_append_paged(
+        _ptr(Kp), _ptr(Vp), _dtype_code(Kp), _ptr(S), _ptr(page_table), max_blocks, num_pages,
+        _ptr(seqlens), _ptr(k_new), _ptr(v_new), batch, Hkv, d, B, _stream(stream)))
+    return Kp, Vp, S, seqlens
+
+
+def ssa_learned_summary(K, qbar, B: int, S=None, stream=None):
+    """Learned block summaries ``[batch, Hkv, N // B, d]`` fp32 (DashAttention's
+    stage 0); ``qbar``: ``[Hkv, d]`` fp32, one learned query per KV head."""
+    _need(K, "K")
+    _need(qbar, "qbar")
+    batch, Hkv, N, d = K.shape
+    if S is None:
+        S = torch.empty(batch, Hkv, N // B, d, dtype=torch.float32, device=K.device)
+    _check("ssa_learned_summary", load_library().ssa_learned_summary(
+        _ptr(K), _dtype_code(K), _ptr(qbar), batch, Hkv, N, d, B, _ptr(S), _stream(stream)))
+    return S
+
+
+def entmax_width(N: int, B: int) -> int:
+    """Row width of ssa_route_entmax's idx / bias: every candidate + the diagonal."""
+    nq, nfull = -(-N // B), N // B
+    return min(nq - 1, nfull) + 1
+
+
+def ssa_route_entmax(Q, S, B: int, Hkv: int, alpha: float, gamma: float, sigma: float,
+                     want_w: bool = False, stream=None):
+    """alpha-entmax routing (DashAttention's stage 1): returns ``(idx, cnt, bias,
+    w)``; ``w`` (``[batch, Hkv, nq, N // B]``) is None unless wanted."""
+    _need(Q, "Q")
+    batch, Hq, N, d = Q.shape
+    nq, nfull = -(-N // B), N // B
+    width = entmax_width(N, B)
+    idx = torch.empty(batch, Hkv, nq, width, dtype=torch.int32, device=Q.device)
+    cnt = torch.empty(batch, Hkv, nq, dtype=torch.int32, device=Q.device)
+    bias = torch.empty(batch, Hkv, nq, width, dtype=torch.float32, device=Q.device)
+    w = torch.empty(batch, Hkv, nq, nfull, dtype=torch.float32, device=Q.device) if want_w else None
+    _check("ssa_route_entmax", load_library().ssa_route_entmax(
+        _ptr(Q), _dtype_code(Q), _ptr(S), batch, Hq, Hkv, N, d, B, ctypes.c_float(alpha),
+        ctypes.c_float(gamma), ctypes.c_float(sigma), width, _ptr(idx), _ptr(cnt), _ptr(bias),
+        _ptr(w), _stream(stream)))
+    return idx, cnt, bias, w
+
+
+def ssa_sparse_attn_fwd_prior(Q, K, V, idx, cnt, bias, B: int, scale: float | None = None,
+                              O=None, lse=None, stream=None):
+    """Attention with the routing prior (DashAttention's stage 2): returns
+    ``(O, lse)``."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (idx, "idx"), (cnt, "cnt"), (bias, "bias")):
+        _need(t, n)
+    batch, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(batch, Hq, N, dtype=torch.float32, device=Q.device)
+    _check("ssa_sparse_attn_fwd_prior", load_library().ssa_sparse_attn_fwd_prior(
+        _ptr(Q), _ptr(K), _ptr(V), _dtype_code(Q), _ptr(idx), _ptr(cnt), _ptr(bias), batch, Hq,
+        Hkv, N, d, B, idx.shape[-1], ctypes.c_float(scale), _ptr(O), _ptr(lse), _stream(stream)))
+    return O, lse
+
+
+def ssa_route_hierarchical(Q, S, B: int, M: int, k_seg: int, k_blk: int, Hkv: int,
+                           idx=None, cnt=None, stream=None):
+    """Two-level routing (segments of ``M`` blocks, then blocks): returns
+    ``(idx, cnt)`` in the layout of ``ssa_route``."""
+    _need(Q, "Q")
+    batch, Hq, N, d = Q.shape
+    nq = -(-N // B)
+    width = min(k_blk, nq) + 2
+    if idx is None:
+        idx = torch.empty(batch, Hkv, nq, width, dtype=torch.int32, device=Q.device)
+    if cnt is None:
+        cnt = torch.empty(batch, Hkv, nq, dtype=torch.int32, device=Q.device)
+    _check("ssa_route_hierarchical", load_library().ssa_route_hierarchical(
+        _ptr(Q), _dtype_code(Q), _ptr(S), batch, Hq, Hkv, N, d, B, M, k_seg, k_blk,
+        idx.shape[-1], _ptr(idx), _ptr(cnt), _stream(stream)))
+    return idx, cnt
+
+
+def ssa_decode_per_head_workspace_size(batch: int, Hq: int, Hkv: int, Lmax: int, d: int, B: int,
+                                       topk: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ssa_decode_per_head_workspace_size",
+           load_library().ssa_decode_per_head_workspace_size(batch, Hq, Hkv, Lmax, d, B, topk,
+                                                             ctypes.byref(n)))
+    return n.value
+
+
+def ssa_decode_per_head(q, Kc, Vc, S, seqlens, B: int, topk: int, scale: float | None = None,
+                        O=None, idx=None, want_idx: bool = True, workspace=None, stream=None):
+    """Decode with one block selection per query head: returns ``(O, idx)``,
+    ``idx`` ``[batch, Hq, width]``."""
+    for t, n in ((q, "q"), (Kc, "Kc"), (Vc, "Vc"), (seqlens, "seqlens")):
+        _need(t, n)
+    batch, Hq, d = q.shape
+    Hkv, Lmax = Kc.shape[1], Kc.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(q)
+    if idx is None and want_idx:
+        idx = torch.empty(batch, Hq, decode_width(Lmax, B, topk), dtype=torch.int32,
+                          device=q.device)
+    nbytes = ssa_decode_per_head_workspace_size(batch, Hq, Hkv, Lmax, d, B, topk)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check("ssa_decode_per_head", load_library().ssa_decode_per_head(
+        _ptr(q), _ptr(Kc), _ptr(Vc), _dtype_code(q), _ptr(S), _ptr(seqlens), batch, Hq, Hkv, Lmax,
+        d, B, topk, ctypes.c_float(scale), _ptr(O), _ptr(idx), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return O, idx
 
 
 def ssa_sparse_attn_bwd(Q, K, V, O, dO, lse, idx, cnt, B: int, scale: float | None = None,

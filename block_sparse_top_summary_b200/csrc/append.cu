@@ -25,7 +25,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(
     T* __restrict__ Kc, T* __restrict__ Vc, float* __restrict__ S, int32_t* __restrict__ seqlens,
     const T* __restrict__ k_new, const T* __restrict__ v_new, int Hkv, int Lmax, int B,
-    int nfull) {
+    int nfull, CacheMap pm) {
   constexpr int EPC = Vec16<T>::n;  // elements per 16-byte chunk
   constexpr int CPR = D / EPC;      // chunks per row
   const int b = blockIdx.x;
@@ -38,15 +38,27 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(
   __syncthreads();
   const int L = s_len;
   if (L < 0 || L >= Lmax) return;  // full cache or invalid length: nothing changes
+  // Paged cache: the page of the block that receives the row.  Every thread
+  // reads the same table word, so the CTA takes one path.
+  int page = -1;
+  if (pm.table != nullptr) {
+    page = pm.table[(int64_t)b * pm.max_blocks + L / B];
+    if (page < 0 || page >= pm.num_pages) return;  // no page for the next block: unchanged
+  }
   const int64_t head0 = (int64_t)b * Hkv;
+  // element offset of row pos of KV head h: contiguous, or row pos % B of the page
+  auto row_at = [&](int h, int pos) -> int64_t {
+    return page < 0 ? ((head0 + h) * Lmax + pos) * D
+                    : (((int64_t)page * Hkv + h) * B + pos % B) * D;
+  };
   // the new rows: chunk w of head h (w < CPR: key, else value)
   for (int e = t; e < Hkv * 2 * CPR; e += kAppendThreads) {
     const int h = e / (2 * CPR), w = e - h * 2 * CPR;
     const int64_t head = head0 + h;
     if (w < CPR) {
-      reinterpret_cast<uint4*>(Kc + (head * Lmax + L) * D)[w] = ldg16(k_new + head * D + w * EPC);
+      reinterpret_cast<uint4*>(Kc + row_at(h, L))[w] = ldg16(k_new + head * D + w * EPC);
     } else {
-      reinterpret_cast<uint4*>(Vc + (head * Lmax + L) * D)[w - CPR] =
+      reinterpret_cast<uint4*>(Vc + row_at(h, L))[w - CPR] =
           ldg16(v_new + head * D + (w - CPR) * EPC);
     }
   }
@@ -67,7 +79,7 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
     const int h = pair / CPR, cc = pair - (pair / CPR) * CPR;
     if (pair < P) {
-      const T* src = Kc + ((head0 + h) * Lmax + (int64_t)j * B) * D + cc * EPC;
+      const T* src = Kc + row_at(h, j * B) + cc * EPC;
 #pragma unroll 8
       for (int r = part; r < B; r += TP) {
         const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src + (int64_t)r * D));
@@ -95,25 +107,25 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(
 template <typename T, int D>
 static cudaError_t launch_append_t(void* Kc, void* Vc, float* S, int32_t* seqlens,
                                    const void* k_new, const void* v_new, int batch, int Hkv,
-                                   int Lmax, int B, cudaStream_t st) {
+                                   int Lmax, int B, cudaStream_t st, CacheMap pm) {
   decode_append_kernel<T, D><<<batch, kAppendThreads, 0, st>>>((T*)Kc, (T*)Vc, S, seqlens, (const T*)k_new,
-                                                    (const T*)v_new, Hkv, Lmax, B, Lmax / B);
+                                                    (const T*)v_new, Hkv, Lmax, B, Lmax / B, pm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_append(void* Kc, void* Vc, ssa_dtype dt, float* S, int32_t* seqlens,
                                  const void* k_new, const void* v_new, int batch, int Hkv,
-                                 int Lmax, int d, int B, cudaStream_t st) {
+                                 int Lmax, int d, int B, cudaStream_t st, CacheMap pm) {
   if (dt == SSA_BF16) {
     return d == 128 ? launch_append_t<__nv_bfloat16, 128>(Kc, Vc, S, seqlens, k_new, v_new, batch,
-                                                          Hkv, Lmax, B, st)
+                                                          Hkv, Lmax, B, st, pm)
                     : launch_append_t<__nv_bfloat16, 64>(Kc, Vc, S, seqlens, k_new, v_new, batch,
-                                                         Hkv, Lmax, B, st);
+                                                         Hkv, Lmax, B, st, pm);
   }
   return d == 128 ? launch_append_t<float, 128>(Kc, Vc, S, seqlens, k_new, v_new, batch, Hkv, Lmax,
-                                                B, st)
+                                                B, st, pm)
                   : launch_append_t<float, 64>(Kc, Vc, S, seqlens, k_new, v_new, batch, Hkv, Lmax,
-                                               B, st);
+                                               B, st, pm);
 }
 
 }  // namespace ssa

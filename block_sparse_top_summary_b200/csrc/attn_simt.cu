@@ -21,9 +21,9 @@ constexpr int KC = 32;  // keys per shared-memory chunk
 template <typename T, int D>
 __global__ void __launch_bounds__(256) attn_simt_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
-    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, T* __restrict__ O,
-    float* __restrict__ lse, int Hq, int Hkv, int N, int B, int nq, int max_sel,
-    float scale_log2) {
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
+    const float* __restrict__ bias, T* __restrict__ O, float* __restrict__ lse, int Hq, int Hkv,
+    int N, int B, int nq, int max_sel, float scale_log2) {
   constexpr int TPR = D / 64;  // threads per row
   constexpr int EPC = Vec16<T>::n;
   constexpr int CPR = D / EPC;
@@ -62,8 +62,11 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(
   const int ns = cnt[(int64_t)(b * Hkv + g) * nq + i];
   const int block_last_row = min(i * B + B, N) - 1;
 
+  const float* brow = bias != nullptr ? bias + ((int64_t)(b * Hkv + g) * nq + i) * max_sel : nullptr;
   for (int s = 0; s < ns; ++s) {
     const int j = sel[s];
+    // prior bias of the block (natural log), in the log2 domain of the logits
+    const float bj = brow != nullptr ? brow[s] * 1.4426950408889634f : 0.f;
     for (int kc = 0; kc < B; kc += KC) {
       const int kb = j * B + kc;
       if (kb > block_last_row) break;  // the rest of this block is in every row's future
@@ -104,7 +107,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(
         // a chunk may reach past block j (B not a multiple of KC): those keys
         // belong to the next block, which this row did not select
         const int kpos = kb + kk;
-        sc[kk] = (kpos <= qpos && kc + kk < B) ? a : -INFINITY;
+        sc[kk] = (kpos <= qpos && kc + kk < B) ? a + bj : -INFINITY;
         cmax = fmaxf(cmax, sc[kk]);
       }
       const float mnew = fmaxf(m, cmax);
@@ -144,30 +147,31 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(
 
 template <typename T, int D>
 static cudaError_t launch_simt_t(const void* Q, const void* K, const void* V, const int32_t* idx,
-                                 const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
-                                 int max_sel, float scale, void* O, float* lse, cudaStream_t st) {
+                                 const int32_t* cnt, const float* bias, int batch, int Hq,
+                                 int Hkv, int N, int B, int max_sel, float scale, void* O,
+                                 float* lse, cudaStream_t st) {
   const int nq = (N + B - 1) / B;
   dim3 grid(nq, batch * Hq);
   const int threads = B * (D / 64);
   attn_simt_kernel<T, D><<<grid, threads, 0, st>>>(
-      (const T*)Q, (const T*)K, (const T*)V, idx, cnt, (T*)O, lse, Hq, Hkv, N, B, nq, max_sel,
-      scale * 1.4426950408889634f);
+      (const T*)Q, (const T*)K, (const T*)V, idx, cnt, bias, (T*)O, lse, Hq, Hkv, N, B, nq,
+      max_sel, scale * 1.4426950408889634f);
   return cudaGetLastError();
 }
 
 cudaError_t launch_attn_simt(const void* Q, const void* K, const void* V, ssa_dtype dt,
-                             const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
-                             int N, int d, int B, int max_sel, float scale, void* O, float* lse,
-                             cudaStream_t st) {
+                             const int32_t* idx, const int32_t* cnt, const float* bias, int batch,
+                             int Hq, int Hkv, int N, int d, int B, int max_sel, float scale,
+                             void* O, float* lse, cudaStream_t st) {
   if (dt == SSA_BF16) {
-    return d == 128 ? launch_simt_t<__nv_bfloat16, 128>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, B,
+    return d == 128 ? launch_simt_t<__nv_bfloat16, 128>(Q, K, V, idx, cnt, bias, batch, Hq, Hkv, N, B,
                                                         max_sel, scale, O, lse, st)
-                    : launch_simt_t<__nv_bfloat16, 64>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, B,
+                    : launch_simt_t<__nv_bfloat16, 64>(Q, K, V, idx, cnt, bias, batch, Hq, Hkv, N, B,
                                                        max_sel, scale, O, lse, st);
   }
-  return d == 128 ? launch_simt_t<float, 128>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, B, max_sel,
+  return d == 128 ? launch_simt_t<float, 128>(Q, K, V, idx, cnt, bias, batch, Hq, Hkv, N, B, max_sel,
                                               scale, O, lse, st)
-                  : launch_simt_t<float, 64>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, B, max_sel,
+                  : launch_simt_t<float, 64>(Q, K, V, idx, cnt, bias, batch, Hq, Hkv, N, B, max_sel,
                                              scale, O, lse, st);
 }
 

@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(256, 2) decode_route_kernel(
     const T* __restrict__ q, const float* __restrict__ S, const int32_t* __restrict__ seqlens,
     int Hq, int Hkv, int Lmax, int B, int nsum, int kk, int width, int32_t* __restrict__ ws_idx,
     int32_t* __restrict__ ws_cnt, int* __restrict__ ws_ctr, int32_t* __restrict__ idx_out,
-    float inv_sqrt_d) {
+    float inv_sqrt_d, int kv_div) {
   constexpr int SL = D / 32;
   extern __shared__ __align__(16) float smem[];
   float* qb = smem;                                          // [D]
@@ -189,7 +189,9 @@ __global__ void __launch_bounds__(256, 2) decode_route_kernel(
     float qs[SL];
 #pragma unroll
     for (int e = 0; e < SL; ++e) qs[e] = qb[lane * SL + e];
-    const float* Sg = S + (int64_t)bg * nsum * D + lane * SL;
+    // the summaries of the unit's cache head (units are query heads when kv_div > 1)
+    const int64_t hc = (int64_t)b * (Hkv / kv_div) + g / kv_div;
+    const float* Sg = S + hc * nsum * D + lane * SL;
     for (int j0 = 1 + warp * 32; j0 <= n; j0 += 32 * 8) {
       float v[32];
 #pragma unroll
@@ -400,7 +402,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
     const int32_t* __restrict__ seqlens, int Hq, int Hkv, int Lmax, int B, int width, int CK,
     int subs, int stages, int stage_bytes, long long U, int parts_max,
     const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
-    float* __restrict__ ws_part, int* __restrict__ ws_ctr, T* __restrict__ O, float scale_log2) {
+    float* __restrict__ ws_part, int* __restrict__ ws_ctr, T* __restrict__ O, float scale_log2,
+    CacheMap pm) {
   using SH = StreamShape<T, D, GP>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ uint64_t full[kMaxStages], empty[kMaxStages];
@@ -449,8 +452,17 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(
       const int k0 = j * B + r * CK;
       const int rr = min(CK, min(L, (j + 1) * B) - k0);
       if (rr <= 0) return;
+      const int b = bg / Hkv, g = bg - b * Hkv;
+      const int Hc = Hkv / pm.kv_div, gc = g / pm.kv_div;  // the cache's head
+      if (pm.table != nullptr) {
+        // the block's page; a missing page reads as an empty unit
+        const int page = j < pm.max_blocks ? pm.table[(int64_t)b * pm.max_blocks + j] : -1;
+        if (page < 0 || page >= pm.num_pages) return;
+        src = (((int64_t)page * Hc + gc) * B + r * CK) * D;
+      } else {
+        src = (((int64_t)b * Hc + gc) * Lmax + k0) * D;
+      }
       rows = rr;
-      src = ((int64_t)bg * Lmax + k0) * D;
     };
     long long src_n;
     int rows_n;
@@ -821,7 +833,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
     int Lmax, int B, int width, int CK, int subs, int stages, long long U, int parts_max,
     const int32_t* __restrict__ ws_idx, const int32_t* __restrict__ ws_cnt,
     float* __restrict__ ws_part, int* __restrict__ ws_ctr, __nv_bfloat16* __restrict__ O,
-    float scale_log2) {
+    float scale_log2, CacheMap pm) {
   constexpr int CKM = 32768 / (4 * D);  // most keys per unit (32 KB of K + V)
   constexpr int NT = CKM / 8;           // S column tiles
   constexpr int KS = D / 16;            // k steps of S
@@ -867,8 +879,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
       ptx::prefetch_tmap(&tmK);
       ptx::prefetch_tmap(&tmV);
     }
-    auto resolve = [&](long long u, int& y, int& rows) {
+    // tensor-map coordinates of a unit: row y, head z (contiguous: z = the
+    // cache head b * Hc + gc; paged: y within the block's page, z = page * Hc
+    // + gc)
+    auto resolve = [&](long long u, int& y, int& z, int& rows) {
       y = 0;
+      z = 0;
       rows = 0;
       if (u >= u1) return;
       const int bg = (int)(u / Ubg);
@@ -880,21 +896,32 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
       const int k0 = j * B + r * CK;
       const int rr = min(CK, min(L, (j + 1) * B) - k0);
       if (rr <= 0) return;
+      const int b = bg / Hkv, g = bg - b * Hkv;
+      const int Hc = Hkv / pm.kv_div, gc = g / pm.kv_div;  // the cache's head
+      if (pm.table != nullptr) {
+        const int page = j < pm.max_blocks ? pm.table[(int64_t)b * pm.max_blocks + j] : -1;
+        if (page < 0 || page >= pm.num_pages) return;
+        y = r * CK;
+        z = page * Hc + gc;
+      } else {
+        y = k0;
+        z = b * Hc + gc;
+      }
       rows = rr;
-      y = k0;
     };
-    int y_n, rows_n;
-    resolve(u0 + lane, y_n, rows_n);
+    int y_n, z_n, rows_n;
+    resolve(u0 + lane, y_n, z_n, rows_n);
     int issued = 0;
     bool ok = true;
     for (int b0 = 0; ok && b0 < nunits; b0 += 32) {
-      const int y_c = y_n, rows_c = rows_n;
-      resolve(u0 + b0 + 32 + lane, y_n, rows_n);
+      const int y_c = y_n, z_c = z_n, rows_c = rows_n;
+      resolve(u0 + b0 + 32 + lane, y_n, z_n, rows_n);
       const int cntb = min(32, nunits - b0);
       for (int i = 0; i < cntb; ++i) {
         const int n = b0 + i;
         const int st = n % stages;
         const int y = __shfl_sync(0xffffffffu, y_c, i);
+        const int z = __shfl_sync(0xffffffffu, z_c, i);
         const int rows = __shfl_sync(0xffffffffu, rows_c, i);
         if (n >= stages && !(ok = warp_wait_bounded(&empty[st], ((n / stages) - 1) & 1, abort)))
           break;
@@ -902,14 +929,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
           info[st] = rows;
           ptx::st_release_s32(&tag[st], n);
           if (rows > 0) {
-            const int bg = (int)((u0 + n) / Ubg);
             unsigned char* dst = base + (size_t)st * stage_bytes;
             // whole boxes land (rows past the sequence are masked, rows past
             // the cache read as zeros), so the byte count is fixed
             ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)stage_bytes);
             for (int bx = 0; bx < NB; ++bx) {
-              ptx::tma_load_3d(dst + bx * CK * 128, &tmK, bx * 64, y, bg, &full[st]);
-              ptx::tma_load_3d(dst + tile_bytes + bx * CK * 128, &tmV, bx * 64, y, bg, &full[st]);
+              ptx::tma_load_3d(dst + bx * CK * 128, &tmK, bx * 64, y, z, &full[st]);
+              ptx::tma_load_3d(dst + tile_bytes + bx * CK * 128, &tmV, bx * 64, y, z, &full[st]);
             }
           } else {
             ptx::mbar_arrive(&full[st]);
@@ -1189,7 +1215,7 @@ template <typename T, int D, int GP>
 static cudaError_t launch_stream(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
                                  const int32_t* seqlens, int batch, int Hq, int Hkv, int Lmax,
                                  int B, float scale, void* O, int32_t* ws_idx, int32_t* ws_cnt,
-                                 int* ws_ctr, float* ws_part, cudaStream_t st) {
+                                 int* ws_ctr, float* ws_part, cudaStream_t st, CacheMap pm) {
   using SH = StreamShape<T, D, GP>;
   const StreamGeom s = stream_geom(batch * Hkv, p.width, D, B, (int)sizeof(T));
   const int stage_bytes = 2 * s.ck * D * (int)sizeof(T);
@@ -1214,7 +1240,7 @@ static cudaError_t launch_stream(const DecodePlan& p, const void* q, const void*
   decode_stream_kernel<T, D, GP><<<(unsigned)grid, kStreamThreads, smem, st>>>(
       (const T*)q, (const T*)Kc, (const T*)Vc, seqlens, Hq, Hkv, Lmax, B, p.width, s.ck, s.subs,
       stages, stage_bytes, s.units, p.parts_max, ws_idx, ws_cnt, ws_part, ws_ctr, (T*)O,
-      scale * 1.4426950408889634f);
+      scale * 1.4426950408889634f, pm);
   return cudaGetLastError();
 }
 
@@ -1222,7 +1248,7 @@ template <int D>
 static cudaError_t launch_mma(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
                               const int32_t* seqlens, int batch, int Hq, int Hkv, int Lmax, int B,
                               float scale, void* O, int32_t* ws_idx, int32_t* ws_cnt, int* ws_ctr,
-                              float* ws_part, cudaStream_t st) {
+                              float* ws_part, cudaStream_t st, CacheMap pm) {
   const StreamGeom s = stream_geom(batch * Hkv, p.width, D, B, 2);
   const int stage_bytes = 4 * s.ck * D;
   const size_t fixed = sizeof(float) * ((size_t)kMmaCW * 8 * D + 2 * (size_t)kMmaCW * 8);
@@ -1232,8 +1258,12 @@ static cudaError_t launch_mma(const DecodePlan& p, const void* q, const void* Kc
   if (stages < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = 1024 + (size_t)stages * stage_bytes + fixed;
   CUtensorMap mk, mv;
-  if (!make_bf16_map(&mk, Kc, D, Lmax, batch * Hkv, s.ck) ||
-      !make_bf16_map(&mv, Vc, D, Lmax, batch * Hkv, s.ck))
+  // contiguous: (d, Lmax, batch * Hkv); paged: (d, B, num_pages * Hkv)
+  const int Hc = Hkv / pm.kv_div;  // the cache's heads
+  const int rows_dim = pm.table != nullptr ? B : Lmax;
+  const int heads_dim = pm.table != nullptr ? pm.num_pages * Hc : batch * Hc;
+  if (!make_bf16_map(&mk, Kc, D, rows_dim, heads_dim, s.ck) ||
+      !make_bf16_map(&mv, Vc, D, rows_dim, heads_dim, s.ck))
     return cudaErrorInvalidValue;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1249,7 +1279,7 @@ static cudaError_t launch_mma(const DecodePlan& p, const void* q, const void* Kc
   decode_mma_kernel<D><<<(unsigned)grid, kMmaThreads, smem, st>>>(
       mk, mv, (const __nv_bfloat16*)q, seqlens, Hq, Hkv, Lmax, B, p.width, s.ck, s.subs, stages,
       s.units, p.parts_max, ws_idx, ws_cnt, ws_part, ws_ctr, (__nv_bfloat16*)O,
-      scale * 1.4426950408889634f);
+      scale * 1.4426950408889634f, pm);
   return cudaGetLastError();
 }
 
@@ -1257,7 +1287,8 @@ template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const void* Kc,
                                    const void* Vc, const float* S, const int32_t* seqlens,
                                    int batch, int Hq, int Hkv, int Lmax, int B, float scale,
-                                   void* O, int32_t* idx_out, void* ws, cudaStream_t st) {
+                                   void* O, int32_t* idx_out, void* ws, cudaStream_t st,
+                                   CacheMap pm) {
   char* w = static_cast<char*>(ws);
   int32_t* ws_idx = reinterpret_cast<int32_t*>(w + p.off_idx);
   int32_t* ws_cnt = reinterpret_cast<int32_t*>(w + p.off_cnt);
@@ -1270,34 +1301,34 @@ static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const voi
   if (e != cudaSuccess) return e;
   decode_route_kernel<T, D><<<batch * Hkv, 256, smem1, st>>>(
       (const T*)q, S, seqlens, Hq, Hkv, Lmax, B, nsum, p.kk, p.width, ws_idx, ws_cnt, ws_ctr,
-      idx_out, 1.0f / sqrtf((float)D));
+      idx_out, 1.0f / sqrtf((float)D), pm.kv_div);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if constexpr (sizeof(T) == 2) {
     return launch_mma<D>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale, O, ws_idx, ws_cnt,
-                         ws_ctr, ws_part, st);
+                         ws_ctr, ws_part, st, pm);
   } else {
     return p.G <= 4 ? launch_stream<T, D, 4>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale,
-                                             O, ws_idx, ws_cnt, ws_ctr, ws_part, st)
+                                             O, ws_idx, ws_cnt, ws_ctr, ws_part, st, pm)
                     : launch_stream<T, D, 8>(p, q, Kc, Vc, seqlens, batch, Hq, Hkv, Lmax, B, scale,
-                                             O, ws_idx, ws_cnt, ws_ctr, ws_part, st);
+                                             O, ws_idx, ws_cnt, ws_ctr, ws_part, st, pm);
   }
 }
 
 cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
                           ssa_dtype dt, const float* S, const int32_t* seqlens, int batch, int Hq,
                           int Hkv, int Lmax, int d, int B, float scale, void* O, int32_t* idx_out,
-                          void* ws, cudaStream_t st) {
+                          void* ws, cudaStream_t st, CacheMap pm) {
   if (dt == SSA_BF16) {
     return d == 128 ? launch_decode_t<__nv_bfloat16, 128>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv,
-                                                          Lmax, B, scale, O, idx_out, ws, st)
+                                                          Lmax, B, scale, O, idx_out, ws, st, pm)
                     : launch_decode_t<__nv_bfloat16, 64>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv,
-                                                         Lmax, B, scale, O, idx_out, ws, st);
+                                                         Lmax, B, scale, O, idx_out, ws, st, pm);
   }
   return d == 128 ? launch_decode_t<float, 128>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv, Lmax, B,
-                                                scale, O, idx_out, ws, st)
+                                                scale, O, idx_out, ws, st, pm)
                   : launch_decode_t<float, 64>(p, q, Kc, Vc, S, seqlens, batch, Hq, Hkv, Lmax, B,
-                                               scale, O, idx_out, ws, st);
+                                               scale, O, idx_out, ws, st, pm);
 }
 
 cudaError_t decode_error_word(int** word) {

@@ -28,9 +28,17 @@ cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const in
                            int max_sel, float scale, void* O, float* lse, cudaStream_t st);
 
 cudaError_t launch_attn_simt(const void* Q, const void* K, const void* V, ssa_dtype dt,
-                             const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
-                             int N, int d, int B, int max_sel, float scale, void* O, float* lse,
-                             cudaStream_t st);
+                             const int32_t* idx, const int32_t* cnt, const float* bias, int batch,
+                             int Hq, int Hkv, int N, int d, int B, int max_sel, float scale,
+                             void* O, float* lse, cudaStream_t st);
+
+// DashAttention's adaptive stages (learned summary, alpha-entmax routing).
+cudaError_t launch_learned_summary(const void* K, ssa_dtype dt, const float* qbar, int batch,
+                                   int Hkv, int N, int d, int B, float* S, cudaStream_t st);
+cudaError_t launch_entmax_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq,
+                                int Hkv, int N, int d, int B, float alpha, float gamma,
+                                float sigma, int max_sel, int32_t* idx, int32_t* cnt,
+                                float* bias, float* w, cudaStream_t st);
 
 // Backward pass of stage 2 (bf16, mma.sync tiles): delta, dQ, dK, dV.
 size_t attn_bwd_smem_bytes(int d, int B);
@@ -39,6 +47,20 @@ cudaError_t launch_attn_bwd(const void* Q, const void* K, const void* V, const v
                             const int32_t* cnt, int batch, int Hq, int Hkv, int N, int d, int B,
                             int max_sel, float scale, void* dQ, void* dK, void* dV, float* delta,
                             cudaStream_t st);
+
+// How the decode kernels address the KV cache.
+// - Paged: page pool [num_pages, Hc, B, d]; table[b * max_blocks + j] is the
+//   page of sequence b's logical block j (-1: none).  table == nullptr means
+//   the contiguous cache [batch, Hc, Lmax, d].
+// - kv_div: the kernels' head units are cache heads (kv_div = 1) or query
+//   heads routed one by one (kv_div = Hq / Hkv): unit head u of sequence b
+//   reads cache head u / kv_div, and Hc = (unit heads) / kv_div.
+struct CacheMap {
+  const int32_t* table = nullptr;
+  int max_blocks = 0;
+  int num_pages = 0;
+  int kv_div = 1;
+};
 
 // Decode: scratch layout and launch.
 struct DecodePlan {
@@ -55,11 +77,16 @@ DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int L
 cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
                           ssa_dtype dt, const float* S, const int32_t* seqlens, int batch, int Hq,
                           int Hkv, int Lmax, int d, int B, float scale, void* O, int32_t* idx_out,
-                          void* ws, cudaStream_t st);
+                          void* ws, cudaStream_t st, CacheMap pm = CacheMap{});
 
 cudaError_t launch_decode_append(void* Kc, void* Vc, ssa_dtype dt, float* S, int32_t* seqlens,
                                  const void* k_new, const void* v_new, int batch, int Hkv,
-                                 int Lmax, int d, int B, cudaStream_t st);
+                                 int Lmax, int d, int B, cudaStream_t st, CacheMap pm = CacheMap{});
+
+// Two-level routing: segments of M complete blocks, then blocks.
+cudaError_t launch_hier_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq,
+                              int Hkv, int N, int d, int B, int M, int k_seg, int k_blk,
+                              int max_sel, int32_t* idx, int32_t* cnt, cudaStream_t st);
 
 // Device error words (one per translation unit that has bounded waits):
 // read and reset; returns the first non-zero code or 0.

@@ -57,7 +57,11 @@ const char* ssa_status_string(int status);
 
 /* Library ABI version (major * 100 + minor).  1.01 added ssa_decode_append,
  * 1.02 ssa_sparse_attn_bwd; 2.00 added the `scores` output of ssa_route (an
- * incompatible signature change) and ssa_check_device_error. */
+ * incompatible signature change) and ssa_check_device_error; 2.01 the paged
+ * cache (ssa_decode_paged, ssa_decode_append_paged); 2.02 DashAttention's
+ * adaptive stages (ssa_learned_summary, ssa_route_entmax,
+ * ssa_sparse_attn_fwd_prior); 2.03 the routing variants (ssa_route_hierarchical,
+ * ssa_decode_per_head, ssa_decode_per_head_workspace_size). */
 int ssa_version(void);
 
 /*
@@ -126,6 +130,91 @@ ssa_status ssa_sparse_attn_fwd(const void* Q, const void* K, const void* V, ssa_
                                const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
                                int N, int d, int B, int max_sel, float scale, void* O, float* lse,
                                ssa_stream stream);
+
+/*
+ * DashAttention's adaptive stages (DashAttention page, "Metodologia").  The
+ * page names alpha-entmax without a formula; it is taken as the standard map
+ *   entmax_alpha(x)_j = [(alpha - 1) x_j - tau]_+ ^ (1 / (alpha - 1)),
+ * tau chosen so that the entries sum to 1 (alpha = 2 is sparsemax).
+ */
+
+/*
+ * Stage 0 with a learned summary query ("Estágio 0": a local attention inside
+ * each block, pooled by one learned query):
+ *   S[b, g, j, :] = sum_t softmax_t(scale * qbar[g] . K[b, g, t]) K[b, g, t, :]
+ * over the B keys t of each complete block j, scale = 1/sqrt(d).  qbar = 0
+ * gives the mean of ssa_block_summary.
+ * K: [batch, Hkv, N, d] of `dtype`; qbar: [Hkv, d] fp32 (one learned query per
+ * KV head); S: [batch, Hkv, nfull, d] fp32 (written).  One warp per block.
+ */
+ssa_status ssa_learned_summary(const void* K, ssa_dtype dtype, const float* qbar, int batch,
+                               int Hkv, int N, int d, int B, float* S, ssa_stream stream);
+
+/*
+ * Stage 1 with alpha-entmax routing ("Estágio 1": each query head scores the
+ * summaries, alpha-entmax turns the scores into sparse routing
+ * probabilities, and the heads of a GQA group average their probabilities so
+ * that they share one support).  For every (b, KV head g, query block i):
+ *   for each query head h of group g: qbar_h = mean of head h's rows of block
+ *     i; z_j = gamma * qbar_h . S[b, g, j] / sqrt(d) for the candidates
+ *     j = 0 .. min(i, nfull) - 1 (the complete blocks before i);
+ *     p_h = entmax_alpha(z) (tau by 40 bisection steps in fp32 on
+ *     [max - 1, max] of (alpha - 1) z);
+ *   w = mean over the group's heads of p_h.
+ * Written per row: idx = the support {j : w_j > 0} ascending, then the
+ * diagonal block i; bias = sigma * ln(w_j) for each support entry and 0 for
+ * the diagonal (the prior of stage 2); cnt = the number of entries; entries
+ * past cnt are -1 (idx) and 0 (bias).  w: NULL, or [batch, Hkv, nq, nfull]
+ * fp32 (written; 0 off the candidates).
+ * idx, bias: [batch, Hkv, nq, max_sel] with max_sel >= min(nq - 1, nfull) + 1.
+ * 1 < alpha <= 8, gamma > 0, sigma >= 0.  One CTA per (b, g, i); its
+ * candidate rows live in shared memory, so nq is limited to about 25000.
+ */
+ssa_status ssa_route_entmax(const void* Q, ssa_dtype dtype, const float* S, int batch, int Hq,
+                            int Hkv, int N, int d, int B, float alpha, float gamma, float sigma,
+                            int max_sel, int32_t* idx, int32_t* cnt, float* bias, float* w,
+                            ssa_stream stream);
+
+/*
+ * Stage 2 with the prior-induced softmax ("Estágio 2": the routing
+ * probabilities act as a prior g ~ w^sigma on the routed keys; the maximiser
+ * of z.p - KL(p || g) is p ~ g exp(z), so a routed key's logit gains
+ * sigma * ln w_j; the diagonal branch has no prior; every other key is
+ * masked).  As ssa_sparse_attn_fwd, with bias[b, g, i, e] added to the scaled
+ * logits of every key of block idx[b, g, i, e] (the causal mask still binds
+ * on the diagonal):
+ *   O[b, h, t] = softmax(scale * q_t . K_sel^T + bias_sel) V_sel.
+ * idx, cnt, bias as written by ssa_route_entmax (bias [batch, Hkv, nq,
+ * max_sel] fp32).  Runs on the CUDA cores (FFMA online softmax).
+ */
+ssa_status ssa_sparse_attn_fwd_prior(const void* Q, const void* K, const void* V,
+                                     ssa_dtype dtype, const int32_t* idx, const int32_t* cnt,
+                                     const float* bias, int batch, int Hq, int Hkv, int N, int d,
+                                     int B, int max_sel, float scale, void* O, float* lse,
+                                     ssa_stream stream);
+
+/*
+ * Two-level routing (Gist Sparse Attention page, "Componentes Principais" 4,
+ * H-GSA: a coarse level over groups of blocks narrows the fine level).
+ * A segment is M consecutive complete blocks (segment m holds blocks mM ..
+ * mM + M - 1); its score is the mean of its blocks' scores, which equals
+ * qbar . (mean of their summaries) / sqrt(d).  For every (b, KV head g, query
+ * block i), with qbar and the block scores s_j of ssa_route:
+ *   - a segment is closed when all its blocks lie before i ((m + 1) M <= i);
+ *     the closed segments holding a candidate compete, and the top k_seg of
+ *     them are kept (equal scores: lower segment index);
+ *   - the pool is the candidates 1 .. i-1 inside a kept segment or inside no
+ *     closed segment (the segment still open at i goes straight to the block
+ *     level, as the diagonal block goes straight to attention);
+ *   - R = the top min(k_blk, pool size) of the pool by s_j (ties: lower
+ *     index); selection = {0} U R U {i}, ascending, -1 padded.
+ * M = 1 with k_seg >= nq is the flat ssa_route.  idx, cnt as for ssa_route,
+ * with max_sel >= min(k_blk, nq) + 2.  k_seg <= 64.  One CTA per (b, g, i).
+ */
+ssa_status ssa_route_hierarchical(const void* Q, ssa_dtype dtype, const float* S, int batch,
+                                  int Hq, int Hkv, int N, int d, int B, int M, int k_seg,
+                                  int k_blk, int max_sel, int32_t* idx, int32_t* cnt,
+                                  ssa_stream stream);
 
 /*
  * Backward pass of stage 2 with the selection held fixed (DashAttention page,
@@ -201,6 +290,27 @@ ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype d
                       size_t ws_bytes, ssa_stream stream);
 
 /*
+ * Decode with per-query-head routing (The Sparse Frontier page, RQ2: in
+ * decode each query can afford its own selection -- Quest selects pages per
+ * query -- while the whole cache stays resident).  As ssa_decode, except that
+ * every query head h routes on its own query instead of the group mean:
+ *   s_j = q[b, h] . S[b, h / G, j] / sqrt(d), j = 1 .. last-1;
+ *   selection_h = {0} U top-k U {last};
+ * and attends only its own selection, reading the cache head h / G.
+ * idx: NULL or [batch, Hq, min(topk, ceil(Lmax / B)) + 2] int32 (written).
+ * workspace: ssa_decode_per_head_workspace_size(...) bytes, 256-byte aligned.
+ * Any G = Hq / Hkv (each unit holds one query row).
+ */
+ssa_status ssa_decode_per_head_workspace_size(int batch, int Hq, int Hkv, int Lmax, int d, int B,
+                                              int topk, size_t* bytes);
+
+ssa_status ssa_decode_per_head(const void* q, const void* Kc, const void* Vc, ssa_dtype dtype,
+                               const float* S, const int32_t* seqlens, int batch, int Hq, int Hkv,
+                               int Lmax, int d, int B, int topk, float scale, void* O,
+                               int32_t* idx, void* workspace, size_t ws_bytes,
+                               ssa_stream stream);
+
+/*
  * Append one token per sequence to the decode KV cache and keep its block
  * summaries current (DashAttention page, "Contribuições Principais" 4,
  * incremental decoding; "Estágio 0": a block's summary is the mean of its B
@@ -227,6 +337,44 @@ ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype d
 ssa_status ssa_decode_append(void* Kc, void* Vc, ssa_dtype dtype, float* S, int32_t* seqlens,
                              const void* k_new, const void* v_new, int batch, int Hkv, int Lmax,
                              int d, int B, ssa_stream stream);
+
+/*
+ * Decode and append over a paged KV cache (The Sparse Frontier page, RQ2:
+ * decode keeps the whole cache and loads only the selected blocks;
+ * DashAttention page, "Contribuições Principais" 4: incremental decoding).
+ * The same computation as ssa_decode / ssa_decode_append on the cache the
+ * page table describes, with no copy into a contiguous cache.
+ *
+ * Layout: a page holds one block of B tokens for every KV head of one
+ * sequence, so the page pools are Kp, Vp: [num_pages, Hkv, B, d] of `dtype`.
+ * page_table: [batch, max_blocks] int32; page_table[b, j] is the page of
+ * logical block j of sequence b, or -1 for none.  Sequences may share pages
+ * (a common prefix).  The cache of sequence b has room for Lmax = max_blocks *
+ * B tokens.  S: [batch, Hkv, max_blocks, d] fp32 block summaries, per sequence
+ * in logical block order.
+ *
+ * ssa_decode_paged: arguments and results as ssa_decode with Lmax =
+ * max_blocks * B (seqlens, O, idx, workspace of ssa_decode_workspace_size for
+ * that Lmax).  Every block that holds tokens of a sequence (j <= (L-1) / B)
+ * must have a page; a selected block without one is skipped (it adds no
+ * keys).  Rows of a page past the sequence's length are never read as keys.
+ *
+ * ssa_decode_append_paged: as ssa_decode_append; the new rows go to row L % B
+ * of page page_table[b, L / B], and a block completed by the append gets its
+ * summary in S[b, :, L / B].  A sequence whose next block has no page is left
+ * unchanged (its length is not raised).
+ * Both: device pointers, 16-byte aligned (the workspace 256-byte aligned).
+ */
+ssa_status ssa_decode_paged(const void* q, const void* Kp, const void* Vp, ssa_dtype dtype,
+                            const float* S, const int32_t* page_table, int max_blocks,
+                            int num_pages, const int32_t* seqlens, int batch, int Hq, int Hkv,
+                            int d, int B, int topk, float scale, void* O, int32_t* idx,
+                            void* workspace, size_t ws_bytes, ssa_stream stream);
+
+ssa_status ssa_decode_append_paged(void* Kp, void* Vp, ssa_dtype dtype, float* S,
+                                   const int32_t* page_table, int max_blocks, int num_pages,
+                                   int32_t* seqlens, const void* k_new, const void* v_new,
+                                   int batch, int Hkv, int d, int B, ssa_stream stream);
 
 /*
  * Largest scratch area ssa_decode_noalloc can use (40 MiB).
