@@ -26,6 +26,11 @@
 // binary search of their ascending index rows, in ascending order, and sums
 // their rows over the G query heads of the group.  No atomics: every output
 // element is written once, in a fixed summation order.
+//
+// Tiles move with 16-byte cp.async copies, all of a thread's copies in flight
+// at once, into two buffers: the next step's tiles (the next selected block's
+// K and V in the dQ pass, the next (query block, head)'s Q, dO, lse and delta
+// in the dK/dV pass) load while the current step's contractions run.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -101,6 +106,43 @@ __device__ __forceinline__ void load_tile(unsigned char* dst, const __nv_bfloat1
   }
 }
 
+// Asynchronous 16-byte (4-byte) copies global -> shared; a source size of 0
+// writes zeros and reads nothing (the address is still a valid one).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int NPEND>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(NPEND) : "memory");
+}
+
+// load_tile with asynchronous copies: every thread's copies are in flight at
+// once; complete them with cp_async_commit / cp_async_wait and a barrier.
+template <int D>
+__device__ __forceinline__ void load_tile_async(uint32_t dst, const __nv_bfloat16* src, int row0,
+                                                int rows, int N) {
+  constexpr int CPR = D / 8;
+  for (int e = threadIdx.x; e < rows * CPR; e += blockDim.x) {
+    const int r = e / CPR, c = e - r * CPR;
+    const bool ok = row0 + r < N;
+    const __nv_bfloat16* p = ok ? src + (size_t)(row0 + r) * D + c * 8 : src;
+    cp_async16(dst + swz<D>(r, c), p, ok ? 16u : 0u);
+  }
+}
+
 }  // namespace
 
 // delta[row] = dO[row] . O[row]; one warp per row, 8 rows per CTA.
@@ -136,12 +178,11 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(
   constexpr int ON = D / 8;       // dQ column tiles
   extern __shared__ __align__(128) unsigned char smem_bwd[];
   const int tile = B * D * 2;
-  unsigned char* sQ = smem_bwd;
-  unsigned char* sG = smem_bwd + tile;  // dO
-  unsigned char* sK = smem_bwd + 2 * tile;
-  unsigned char* sV = smem_bwd + 3 * tile;
-  const uint32_t aQ = ptx::smem_u32(sQ), aG = ptx::smem_u32(sG);
-  const uint32_t aK = ptx::smem_u32(sK), aV = ptx::smem_u32(sV);
+  // Q, dO, then K and V twice: the next selected block's tiles load while
+  // the current one is in use
+  const uint32_t aQ = ptx::smem_u32(smem_bwd), aG = aQ + tile;
+  auto k_at = [&](int buf) { return aQ + (uint32_t)((2 + 2 * buf) * tile); };
+  auto v_at = [&](int buf) { return aQ + (uint32_t)((3 + 2 * buf) * tile); };
 
   const int i = blockIdx.x % nq;
   const int bh = blockIdx.x / nq;  // b * Hq + h
@@ -153,8 +194,8 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(
   const size_t hoff = (size_t)bh * N * D;
   const size_t goff = ((size_t)b * Hkv + g) * N * D;
 
-  load_tile<D>(sQ, Q + hoff, q0, B, N);
-  load_tile<D>(sG, dO + hoff, q0, B, N);
+  load_tile_async<D>(aQ, Q + hoff, q0, B, N);
+  load_tile_async<D>(aG, dO + hoff, q0, B, N);
 
   // this lane's two query rows: warp * 16 + gr and + 8
   const int ra = q0 + warp * 16 + gr, rb = ra + 8;
@@ -171,13 +212,31 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(
   const size_t urow = ((size_t)b * Hkv + g) * nq + i;
   const int n_sel = min(max(cnt[urow], 0), max_sel);
   const int32_t* sel = idx + urow * max_sel;
-  for (int s = 0; s < n_sel; ++s) {
+  // entries outside [0, i] are skipped (the same for every thread)
+  auto next_valid = [&](int s) {
+    while (s < n_sel && (sel[s] < 0 || sel[s] > i)) ++s;
+    return s;
+  };
+  int s = next_valid(0);
+  if (s < n_sel) {
+    load_tile_async<D>(k_at(0), K + goff, sel[s] * B, B, N);
+    load_tile_async<D>(v_at(0), V + goff, sel[s] * B, B, N);
+  }
+  cp_async_commit();  // group: Q, dO and the first K / V
+  for (int it = 0; s < n_sel; ++it) {
     const int j = sel[s];
-    if (j < 0 || j > i) continue;  // uniform over the CTA
-    __syncthreads();               // the previous K / V tiles are consumed
-    load_tile<D>(sK, K + goff, j * B, B, N);
-    load_tile<D>(sV, V + goff, j * B, B, N);
+    const int buf = it & 1;
+    const int s2 = next_valid(s + 1);
+    __syncthreads();  // the other buffer's tiles (previous block) are consumed
+    if (s2 < n_sel) {
+      load_tile_async<D>(k_at(buf ^ 1), K + goff, sel[s2] * B, B, N);
+      load_tile_async<D>(v_at(buf ^ 1), V + goff, sel[s2] * B, B, N);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();  // everything but the newest group has landed
     __syncthreads();
+    s = s2;
+    const uint32_t aK = k_at(buf), aV = v_at(buf);
     for (int kc = 0; kc < B; kc += CH) {
       const int nk = min(CH, B - kc);  // a multiple of 16
       float sc[NT][4], dp[NT][4];
@@ -237,6 +296,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dq_kernel(
       }
     }
   }
+  cp_async_wait<0>();  // no copy outlives the CTA
   // dQ = scale * acc, rows past N skipped
 #pragma unroll
   for (int n = 0; n < ON; ++n) {
@@ -265,16 +325,15 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
   constexpr int ON = D / 8;
   extern __shared__ __align__(128) unsigned char smem_bwd[];
   const int tile = B * D * 2;
-  unsigned char* sK = smem_bwd;
-  unsigned char* sV = smem_bwd + tile;
-  unsigned char* sQ = smem_bwd + 2 * tile;
-  unsigned char* sG = smem_bwd + 3 * tile;  // dO
-  float* s_lse = reinterpret_cast<float*>(smem_bwd + 4 * tile);  // [B], log2 units
-  float* s_del = s_lse + B;                                      // [B]
+  // K, V, then Q and dO twice (the next step's tiles load while the current
+  // ones are in use), then lse and delta twice ([2][B] each, natural log)
+  const uint32_t aK = ptx::smem_u32(smem_bwd), aV = aK + tile;
+  auto q_at = [&](int buf) { return aK + (uint32_t)((2 + 2 * buf) * tile); };
+  auto g_at = [&](int buf) { return aK + (uint32_t)((3 + 2 * buf) * tile); };
+  float* s_lse = reinterpret_cast<float*>(smem_bwd + 6 * tile);
+  float* s_del = s_lse + 2 * B;
   __shared__ int s_list[256];
   __shared__ int s_wcnt[8];
-  const uint32_t aK = ptx::smem_u32(sK), aV = ptx::smem_u32(sV);
-  const uint32_t aQ = ptx::smem_u32(sQ), aG = ptx::smem_u32(sG);
 
   const int nbg = batch * Hkv;
   const int j = blockIdx.x / nbg;  // key block first: the sink column runs in the first wave
@@ -287,8 +346,27 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
   const size_t goff = (size_t)bg * N * D;
   const float c2 = scale * kLog2e;
 
-  load_tile<D>(sK, K + goff, j * B, B, N);
-  load_tile<D>(sV, V + goff, j * B, B, N);
+  load_tile_async<D>(aK, K + goff, j * B, B, N);
+  load_tile_async<D>(aV, V + goff, j * B, B, N);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // step stp of a range: hit stp / G, head stp % G, into buffer buf
+  auto issue = [&](int stp, int buf) {
+    const int i = s_list[stp / G];
+    const int bh = b * Hq + g * G + stp % G;
+    load_tile_async<D>(q_at(buf), Q + (size_t)bh * N * D, i * B, B, N);
+    load_tile_async<D>(g_at(buf), dO + (size_t)bh * N * D, i * B, B, N);
+    for (int r = threadIdx.x; r < B; r += blockDim.x) {
+      const int t = i * B + r;
+      const bool ok = t < N;
+      cp_async4(ptx::smem_u32(s_lse + buf * B + r), ok ? lse + (size_t)bh * N + t : lse,
+                ok ? 4u : 0u);
+      cp_async4(ptx::smem_u32(s_del + buf * B + r), ok ? delta + (size_t)bh * N + t : delta,
+                ok ? 4u : 0u);
+    }
+  };
 
   float dk[ON][4], dv[ON][4];
 #pragma unroll
@@ -331,20 +409,21 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
     if (hit) s_list[off + __popc(bal & ((1u << lane) - 1u))] = qi;
     __syncthreads();
 
-    for (int li = 0; li < n_hit; ++li) {
-      const int i = s_list[li];
-      for (int hh = 0; hh < G; ++hh) {
-        const int bh = b * Hq + g * G + hh;
-        const size_t hoff = (size_t)bh * N * D;
-        __syncthreads();  // the previous Q / dO tiles are consumed
-        load_tile<D>(sQ, Q + hoff, i * B, B, N);
-        load_tile<D>(sG, dO + hoff, i * B, B, N);
-        for (int r = threadIdx.x; r < B; r += blockDim.x) {
-          const int t = i * B + r;
-          s_lse[r] = t < N ? lse[(size_t)bh * N + t] * kLog2e : INFINITY;
-          s_del[r] = t < N ? delta[(size_t)bh * N + t] : 0.f;
-        }
-        __syncthreads();
+    const int nst = n_hit * G;
+    if (nst > 0) issue(0, 0);
+    cp_async_commit();
+    for (int stp = 0; stp < nst; ++stp) {
+      const int buf = stp & 1;
+      __syncthreads();  // the other buffer (previous step) is consumed
+      if (stp + 1 < nst) issue(stp + 1, buf ^ 1);
+      cp_async_commit();
+      cp_async_wait<1>();  // this step's group has landed
+      __syncthreads();
+      {
+        const int i = s_list[stp / G];
+        const uint32_t aQ = q_at(buf), aG = g_at(buf);
+        const float* lse_b = s_lse + buf * B;
+        const float* del_b = s_del + buf * B;
         for (int qc = 0; qc < B; qc += CH) {
           const int nqc = min(CH, B - qc);  // a multiple of 16
           float st[NT][4], dpt[NT][4];  // S^T and dP^T: this warp's 16 keys x the chunk's queries
@@ -381,9 +460,9 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
               const int ql = qc + n * 8 + 2 * tq + (e & 1);  // query within block i
               const int key = e < 2 ? ka : kb_;
               float p = 0.f, ds = 0.f;
-              if (ql < B && key <= i * B + ql) {
-                p = exp2f(fmaf(st[n][e], c2, -s_lse[ql]));
-                ds = p * (dpt[n][e] - s_del[ql]);
+              if (ql < B && key <= i * B + ql && i * B + ql < N) {
+                p = exp2f(fmaf(st[n][e], c2, -lse_b[ql] * kLog2e));
+                ds = p * (dpt[n][e] - del_b[ql]);
               }
               st[n][e] = p;
               dpt[n][e] = ds;
@@ -413,6 +492,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
     }
     __syncthreads();  // s_wcnt and s_list are rewritten by the next range
   }
+  cp_async_wait<0>();  // no copy outlives the CTA
   // dK = scale * dk, dV = dv; key rows past N skipped
 #pragma unroll
   for (int n = 0; n < ON; ++n) {
@@ -433,7 +513,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
 }
 
 size_t attn_bwd_smem_bytes(int d, int B) {
-  return (size_t)4 * B * d * 2 + (size_t)2 * B * sizeof(float);
+  return (size_t)6 * B * d * 2 + (size_t)4 * B * sizeof(float);
 }
 
 template <int D>
