@@ -493,11 +493,13 @@ def run_ours(args, world, rank, local):
     dOd = upstream_grad(c32.batch, c32.Hq, c32.N, c32.d, seed=rank_seed(c32.seed + 1, rank),
                         dtype=c32.dtype, device=dev)
     dQb, dKb, dVb = torch.empty_like(p32.Q), torch.empty_like(p32.K), torch.empty_like(p32.V)
-    delta = torch.empty(c32.batch, c32.Hq, c32.N, dtype=torch.float32, device=dev)
+    bws = torch.empty(ssa.ssa_sparse_attn_bwd_workspace_size(c32.batch, c32.Hq, c32.Hkv, c32.N,
+                                                             c32.d, c32.B),
+                      dtype=torch.uint8, device=dev)
 
     def bwd():
         ssa.ssa_sparse_attn_bwd(p32.Q, p32.K, p32.V, p32.O, dOd, p32.lse, p32.idx, p32.cnt,
-                                c32.B, dQ=dQb, dK=dKb, dV=dVb, delta=delta)
+                                c32.B, dQ=dQb, dK=dKb, dV=dVb, workspace=bws)
 
     bwd_ms = []
     for it in range(2 + 5):

@@ -29,6 +29,7 @@ from .abi import (  # noqa: F401
     ssa_sparse_attn_fwd_prior,
     ssa_route,
     ssa_sparse_attn_bwd,
+    ssa_sparse_attn_bwd_workspace_size,
     ssa_sparse_attn_fwd,
     ssa_sparse_attn_uses_tensor_cores,
 )

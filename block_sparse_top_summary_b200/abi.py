@@ -29,6 +29,7 @@ EXPORTS = ("ssa_status_string", "ssa_version", "ssa_block_summary", "ssa_route",
            "ssa_decode_paged", "ssa_decode_append_paged", "ssa_learned_summary",
            "ssa_route_entmax", "ssa_sparse_attn_fwd_prior", "ssa_route_hierarchical",
            "ssa_decode_per_head", "ssa_decode_per_head_workspace_size",
+           "ssa_sparse_attn_bwd_workspace_size",
            "ssa_device_error", "ssa_check_device_error", "ssa_debug_wait_timeout")
 
 
@@ -66,7 +67,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.ssa_decode_noalloc.argtypes = [vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f, vp, vp, vp]
     lib.ssa_decode_append.argtypes = [vp, vp, i, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.ssa_sparse_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, i, i, i, i, i, f,
-                                        vp, vp, vp, vp, vp]
+                                        vp, vp, vp, vp, sz, vp]
+    lib.ssa_sparse_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i, ctypes.POINTER(sz)]
     lib.ssa_debug_wait_timeout.argtypes = [i, vp]
     lib.ssa_decode_paged.argtypes = [vp, vp, vp, i, vp, vp, i, i, vp, i, i, i, i, i, i, f, vp, vp,
                                      vp, sz, vp]
@@ -449,18 +451,27 @@ def ssa_decode_per_head(q, Kc, Vc, S, seqlens, B: int, topk: int, scale: float |
     return O, idx
 
 
+def ssa_sparse_attn_bwd_workspace_size(batch: int, Hq: int, Hkv: int, N: int, d: int,
+                                       B: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("ssa_sparse_attn_bwd_workspace_size",
+           load_library().ssa_sparse_attn_bwd_workspace_size(batch, Hq, Hkv, N, d, B,
+                                                            ctypes.byref(n)))
+    return n.value
+
+
 def ssa_sparse_attn_bwd(Q, K, V, O, dO, lse, idx, cnt, B: int, scale: float | None = None,
-                        dQ=None, dK=None, dV=None, delta=None, stream=None):
+                        dQ=None, dK=None, dV=None, workspace=None, stream=None):
     """Gradients of the selected-block attention: returns ``(dQ, dK, dV)``.
 
     ``O`` and ``lse`` are the outputs of ``ssa_sparse_attn_fwd`` on the same
     ``Q, K, V, idx, cnt``; ``dO`` is the gradient of the loss with respect to
-    ``O``.  ``delta`` (``[batch, Hq, N]`` fp32) is scratch.
+    ``O``.  ``workspace`` (uint8, ``ssa_sparse_attn_bwd_workspace_size`` bytes)
+    is scratch.
     """
     for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O"), (dO, "dO"), (lse, "lse"), (idx, "idx"),
                  (cnt, "cnt")):
         _need(t, n)
-    fn = load_library().ssa_sparse_attn_bwd
     batch, Hq, N, d = Q.shape
     Hkv = K.shape[1]
     if scale is None:
@@ -468,12 +479,14 @@ def ssa_sparse_attn_bwd(Q, K, V, O, dO, lse, idx, cnt, B: int, scale: float | No
     dQ = torch.empty_like(Q) if dQ is None else dQ
     dK = torch.empty_like(K) if dK is None else dK
     dV = torch.empty_like(V) if dV is None else dV
-    if delta is None:
-        delta = torch.empty(batch, Hq, N, dtype=torch.float32, device=Q.device)
-    _check("ssa_sparse_attn_bwd", fn(
+    if workspace is None:
+        workspace = torch.empty(ssa_sparse_attn_bwd_workspace_size(batch, Hq, Hkv, N, d, B),
+                                dtype=torch.uint8, device=Q.device)
+    _check("ssa_sparse_attn_bwd", load_library().ssa_sparse_attn_bwd(
         _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(lse), _dtype_code(Q), _ptr(idx),
         _ptr(cnt), batch, Hq, Hkv, N, d, B, idx.shape[-1], ctypes.c_float(scale), _ptr(dQ),
-        _ptr(dK), _ptr(dV), _ptr(delta), _stream(stream)))
+        _ptr(dK), _ptr(dV), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
     return dQ, dK, dV
 
 

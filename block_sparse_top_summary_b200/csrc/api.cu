@@ -56,7 +56,7 @@ const char* ssa_status_string(int status) {
   }
 }
 
-int ssa_version(void) { return 203; }
+int ssa_version(void) { return 204; }
 
 ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv, int N, int d,
                              int B, float* S, ssa_stream stream) {
@@ -165,11 +165,21 @@ ssa_status ssa_sparse_attn_fwd_prior(const void* Q, const void* K, const void* V
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
+ssa_status ssa_sparse_attn_bwd_workspace_size(int batch, int Hq, int Hkv, int N, int d, int B,
+                                              size_t* bytes) {
+  if (bytes == nullptr) return SSA_ERR_INVALID_ARG;
+  ssa_status st = check_dims(d, B, SSA_BF16);
+  if (st != SSA_OK) return st;
+  if (batch <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
+  *bytes = ssa::plan_bwd(batch, Hq, Hkv, N, d, B).bytes;
+  return SSA_OK;
+}
+
 ssa_status ssa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O,
                                const void* dO, const float* lse, ssa_dtype dtype,
                                const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
                                int N, int d, int B, int max_sel, float scale, void* dQ, void* dK,
-                               void* dV, float* delta, ssa_stream stream) {
+                               void* dV, void* workspace, size_t ws_bytes, ssa_stream stream) {
   ssa_status st = check_dims(d, B, dtype);
   if (st != SSA_OK) return st;
   if (dtype != SSA_BF16) return SSA_ERR_UNSUPPORTED;
@@ -178,16 +188,19 @@ ssa_status ssa_sparse_attn_bwd(const void* Q, const void* K, const void* V, cons
   if (!(scale > 0.f)) return SSA_ERR_INVALID_ARG;
   if (Q == nullptr || K == nullptr || V == nullptr || O == nullptr || dO == nullptr ||
       lse == nullptr || idx == nullptr || cnt == nullptr || dQ == nullptr || dK == nullptr ||
-      dV == nullptr || delta == nullptr)
+      dV == nullptr || workspace == nullptr)
     return SSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
       !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
     return SSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSA_ERR_INVALID_ARG;
   const long long nq = ((long long)N + B - 1) / B;
   if ((long long)batch * Hq * nq > 0x7fffffffLL || (long long)batch * Hq * N / 8 > 0x7fffffffLL)
     return SSA_ERR_UNSUPPORTED;
-  return from_cuda(ssa::launch_attn_bwd(Q, K, V, O, dO, lse, idx, cnt, batch, Hq, Hkv, N, d, B,
-                                        max_sel, scale, dQ, dK, dV, delta,
+  const ssa::BwdPlan pl = ssa::plan_bwd(batch, Hq, Hkv, N, d, B);
+  if (ws_bytes < pl.bytes) return SSA_ERR_INVALID_ARG;
+  return from_cuda(ssa::launch_attn_bwd(pl, Q, K, V, O, dO, lse, idx, cnt, batch, Hq, Hkv, N, d,
+                                        B, max_sel, scale, dQ, dK, dV, workspace,
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 

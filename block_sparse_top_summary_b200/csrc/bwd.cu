@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
     const float* __restrict__ lse, const float* __restrict__ delta,
     const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int batch, int Hq, int Hkv,
     int N, int B, int nq, int max_sel, float scale, __nv_bfloat16* __restrict__ dK,
-    __nv_bfloat16* __restrict__ dV) {
+    __nv_bfloat16* __restrict__ dV, float* __restrict__ sink_part, int sink_qr, int sink_nsplit) {
   constexpr int CH = chunk_of<D>();
   constexpr int NT = CH / 8;  // query column tiles per chunk
   constexpr int KS = D / 16;
@@ -336,8 +336,26 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
   __shared__ int s_wcnt[8];
 
   const int nbg = batch * Hkv;
-  const int j = blockIdx.x / nbg;  // key block first: the sink column runs in the first wave
-  const int bg = blockIdx.x - j * nbg;
+  // CTAs [0, nbg * sink_nsplit) take the sink column (key block 0, which every
+  // query block selects) in ranges of sink_qr query blocks and write fp32
+  // partial sums; the others take one key block j >= 1 each over every query
+  // block i >= j.  The sink ranges come first, so they start in the first wave.
+  const int nsink = nbg * sink_nsplit;
+  const bool sink = (int)blockIdx.x < nsink;
+  int j, bg, i_lo, i_hi;
+  if (sink) {
+    const int rg = blockIdx.x / nbg;
+    j = 0;
+    bg = blockIdx.x - rg * nbg;
+    i_lo = rg * sink_qr;
+    i_hi = min(nq, i_lo + sink_qr);
+  } else {
+    const int u = blockIdx.x - nsink;
+    j = 1 + u / nbg;
+    bg = u - (j - 1) * nbg;
+    i_lo = j;
+    i_hi = nq;
+  }
   const int b = bg / Hkv, g = bg - b * Hkv;
   const int G = Hq / Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -379,11 +397,11 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
   const int32_t* idx_bg = idx + (size_t)bg * nq * max_sel;
   const int32_t* cnt_bg = cnt + (size_t)bg * nq;
 
-  for (int base = j; base < nq; base += blockDim.x) {
+  for (int base = i_lo; base < i_hi; base += blockDim.x) {
     // ---- the query blocks in [base, base + blockDim.x) whose selection holds j
     const int qi = base + threadIdx.x;
     bool hit = false;
-    if (qi < nq) {
+    if (qi < i_hi) {
       const int32_t* row = idx_bg + (size_t)qi * max_sel;
       int lo = 0, hi = min(max(cnt_bg[qi], 0), max_sel);  // ascending entries in [lo, hi)
       while (lo < hi) {
@@ -493,6 +511,21 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
     __syncthreads();  // s_wcnt and s_list are rewritten by the next range
   }
   cp_async_wait<0>();  // no copy outlives the CTA
+  if (sink) {
+    // fp32 partial sums of this range: [range][bg][dK, dV][B][D], unscaled
+    float* pk = sink_part + ((size_t)(blockIdx.x / nbg) * nbg + bg) * 2 * B * D;
+    float* pv = pk + (size_t)B * D;
+    const int ra = warp * 16 + gr, rb = ra + 8;
+#pragma unroll
+    for (int n = 0; n < ON; ++n) {
+      const int col = n * 8 + 2 * tq;
+      *reinterpret_cast<float2*>(pk + (size_t)ra * D + col) = make_float2(dk[n][0], dk[n][1]);
+      *reinterpret_cast<float2*>(pv + (size_t)ra * D + col) = make_float2(dv[n][0], dv[n][1]);
+      *reinterpret_cast<float2*>(pk + (size_t)rb * D + col) = make_float2(dk[n][2], dk[n][3]);
+      *reinterpret_cast<float2*>(pv + (size_t)rb * D + col) = make_float2(dv[n][2], dv[n][3]);
+    }
+    return;
+  }
   // dK = scale * dk, dV = dv; key rows past N skipped
 #pragma unroll
   for (int n = 0; n < ON; ++n) {
@@ -512,18 +545,57 @@ __global__ void __launch_bounds__(256, 1) bwd_dkv_kernel(
   }
 }
 
+// dK and dV of the sink block: the ranges' partial sums added in range order
+// (a fixed order: the result does not depend on scheduling), dK scaled.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_sink_reduce_kernel(
+    const float* __restrict__ sink_part, int nbg, int nsplit, int B, int N, float scale,
+    __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV) {
+  const int bg = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;  // element of the B x D tile
+  if (e >= B * D) return;
+  const int r = e / D;
+  float k = 0.f, v = 0.f;
+  for (int rg = 0; rg < nsplit; ++rg) {
+    const float* p = sink_part + ((size_t)rg * nbg + bg) * 2 * B * D;
+    k += p[e];
+    v += p[(size_t)B * D + e];
+  }
+  if (r < N) {
+    dK[(size_t)bg * N * D + e] = __float2bfloat16_rn(k * scale);
+    dV[(size_t)bg * N * D + e] = __float2bfloat16_rn(v);
+  }
+}
+
 size_t attn_bwd_smem_bytes(int d, int B) {
   return (size_t)6 * B * d * 2 + (size_t)4 * B * sizeof(float);
 }
 
-template <int D>
-static cudaError_t launch_bwd_t(const void* Q, const void* K, const void* V, const void* O,
-                                const void* dO, const float* lse, const int32_t* idx,
-                                const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
-                                int max_sel, float scale, void* dQ, void* dK, void* dV,
-                                float* delta, cudaStream_t st) {
-  using bf = __nv_bfloat16;
+BwdPlan plan_bwd(int batch, int Hq, int Hkv, int N, int d, int B) {
+  BwdPlan p{};
   const int nq = (N + B - 1) / B;
+  const int G = Hq / Hkv;
+  p.sink_qr = 256 / G > 16 ? 256 / G : 16;  // about 256 (query block, head) steps per range
+  p.sink_nsplit = (nq + p.sink_qr - 1) / p.sink_qr;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  p.off_delta = 0;
+  p.off_part = up((size_t)batch * Hq * N * sizeof(float));
+  p.bytes = up(p.off_part +
+               (size_t)batch * Hkv * p.sink_nsplit * 2 * (size_t)B * d * sizeof(float));
+  return p;
+}
+
+template <int D>
+static cudaError_t launch_bwd_t(const BwdPlan& pl, const void* Q, const void* K, const void* V,
+                                const void* O, const void* dO, const float* lse,
+                                const int32_t* idx, const int32_t* cnt, int batch, int Hq,
+                                int Hkv, int N, int B, int max_sel, float scale, void* dQ,
+                                void* dK, void* dV, void* ws, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.off_delta);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + pl.off_part);
+  const int nq = (N + B - 1) / B;
+  const int nbg = batch * Hkv;
   const long long rows = (long long)batch * Hq * N;
   const unsigned threads = (unsigned)(2 * B);  // B / 16 warps
   const size_t smem = attn_bwd_smem_bytes(D, B);
@@ -542,22 +614,28 @@ static cudaError_t launch_bwd_t(const void* Q, const void* K, const void* V, con
   e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  bwd_dkv_kernel<D><<<(unsigned)((long long)batch * Hkv * nq), threads, smem, st>>>(
+  const long long ctas = (long long)nbg * pl.sink_nsplit + (long long)nbg * (nq - 1);
+  bwd_dkv_kernel<D><<<(unsigned)ctas, threads, smem, st>>>(
       (const bf*)Q, (const bf*)K, (const bf*)V, (const bf*)dO, lse, delta, idx, cnt, batch, Hq,
-      Hkv, N, B, nq, max_sel, scale, (bf*)dK, (bf*)dV);
+      Hkv, N, B, nq, max_sel, scale, (bf*)dK, (bf*)dV, part, pl.sink_qr, pl.sink_nsplit);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 rgrid((unsigned)((B * D + 255) / 256), (unsigned)nbg);
+  bwd_sink_reduce_kernel<D><<<rgrid, 256, 0, st>>>(part, nbg, pl.sink_nsplit, B, N, scale,
+                                                   (bf*)dK, (bf*)dV);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_bwd(const void* Q, const void* K, const void* V, const void* O,
-                            const void* dO, const float* lse, const int32_t* idx,
+cudaError_t launch_attn_bwd(const BwdPlan& pl, const void* Q, const void* K, const void* V,
+                            const void* O, const void* dO, const float* lse, const int32_t* idx,
                             const int32_t* cnt, int batch, int Hq, int Hkv, int N, int d, int B,
-                            int max_sel, float scale, void* dQ, void* dK, void* dV, float* delta,
+                            int max_sel, float scale, void* dQ, void* dK, void* dV, void* ws,
                             cudaStream_t st) {
   if (d == 128)
-    return launch_bwd_t<128>(Q, K, V, O, dO, lse, idx, cnt, batch, Hq, Hkv, N, B, max_sel, scale,
-                             dQ, dK, dV, delta, st);
-  return launch_bwd_t<64>(Q, K, V, O, dO, lse, idx, cnt, batch, Hq, Hkv, N, B, max_sel, scale, dQ,
-                          dK, dV, delta, st);
+    return launch_bwd_t<128>(pl, Q, K, V, O, dO, lse, idx, cnt, batch, Hq, Hkv, N, B, max_sel,
+                             scale, dQ, dK, dV, ws, st);
+  return launch_bwd_t<64>(pl, Q, K, V, O, dO, lse, idx, cnt, batch, Hq, Hkv, N, B, max_sel, scale,
+                          dQ, dK, dV, ws, st);
 }
 
 }  // namespace ssa

@@ -40,12 +40,20 @@ cudaError_t launch_entmax_route(const void* Q, ssa_dtype dt, const float* S, int
                                 float sigma, int max_sel, int32_t* idx, int32_t* cnt,
                                 float* bias, float* w, cudaStream_t st);
 
-// Backward pass of stage 2 (bf16, mma.sync tiles): delta, dQ, dK, dV.
+// Backward pass of stage 2 (bf16, mma.sync tiles): delta, dQ, dK, dV.  The
+// workspace holds delta ([batch, Hq, N] fp32) and the sink column's partial
+// sums ([sink_nsplit][batch * Hkv][2][B][d] fp32).
+struct BwdPlan {
+  int sink_qr;      // query blocks per sink range
+  int sink_nsplit;  // sink ranges per (batch, KV head)
+  size_t off_delta, off_part, bytes;
+};
+BwdPlan plan_bwd(int batch, int Hq, int Hkv, int N, int d, int B);
 size_t attn_bwd_smem_bytes(int d, int B);
-cudaError_t launch_attn_bwd(const void* Q, const void* K, const void* V, const void* O,
-                            const void* dO, const float* lse, const int32_t* idx,
+cudaError_t launch_attn_bwd(const BwdPlan& pl, const void* Q, const void* K, const void* V,
+                            const void* O, const void* dO, const float* lse, const int32_t* idx,
                             const int32_t* cnt, int batch, int Hq, int Hkv, int N, int d, int B,
-                            int max_sel, float scale, void* dQ, void* dK, void* dV, float* delta,
+                            int max_sel, float scale, void* dQ, void* dK, void* dV, void* ws,
                             cudaStream_t st);
 
 // How the decode kernels address the KV cache.

@@ -61,7 +61,9 @@ const char* ssa_status_string(int status);
  * cache (ssa_decode_paged, ssa_decode_append_paged); 2.02 DashAttention's
  * adaptive stages (ssa_learned_summary, ssa_route_entmax,
  * ssa_sparse_attn_fwd_prior); 2.03 the routing variants (ssa_route_hierarchical,
- * ssa_decode_per_head, ssa_decode_per_head_workspace_size). */
+ * ssa_decode_per_head, ssa_decode_per_head_workspace_size); 2.04 the backward
+ * takes a sized workspace (ssa_sparse_attn_bwd_workspace_size) in place of
+ * its delta scratch. */
 int ssa_version(void);
 
 /*
@@ -237,7 +239,12 @@ ssa_status ssa_route_hierarchical(const void* Q, ssa_dtype dtype, const float* S
  * Q, O, dO, dQ: [batch, Hq, N, d]; K, V, dK, dV: [batch, Hkv, N, d]; all bf16
  * (SSA_ERR_UNSUPPORTED for SSA_F32).  lse: [batch, Hq, N] fp32 as written by
  * ssa_sparse_attn_fwd; idx/cnt: as written by ssa_route (ascending entries).
- * delta: caller-owned fp32 scratch of batch * Hq * N floats (overwritten).
+ * workspace: caller-owned device scratch of at least
+ * ssa_sparse_attn_bwd_workspace_size(...) bytes, 256-byte aligned, contents on
+ * entry ignored.  It holds delta and the partial sums of the sink block
+ * (block 0, which every query block selects): its dK and dV are summed over
+ * ranges of query blocks by separate CTAs, and the ranges are added in a
+ * fixed order.  Calls that share a workspace must not overlap on the device.
  * The contractions run on mma.sync tensor-core tiles (bf16 in, fp32
  * accumulate); P and dS are rounded to bf16 as operands, outputs to bf16.
  */
@@ -245,7 +252,11 @@ ssa_status ssa_sparse_attn_bwd(const void* Q, const void* K, const void* V, cons
                                const void* dO, const float* lse, ssa_dtype dtype,
                                const int32_t* idx, const int32_t* cnt, int batch, int Hq, int Hkv,
                                int N, int d, int B, int max_sel, float scale, void* dQ, void* dK,
-                               void* dV, float* delta, ssa_stream stream);
+                               void* dV, void* workspace, size_t ws_bytes, ssa_stream stream);
+
+/* Scratch size, in bytes, that ssa_sparse_attn_bwd needs for these sizes. */
+ssa_status ssa_sparse_attn_bwd_workspace_size(int batch, int Hq, int Hkv, int N, int d, int B,
+                                              size_t* bytes);
 
 /*
  * 1 if ssa_sparse_attn_fwd runs this shape on the tensor cores, else 0 (the

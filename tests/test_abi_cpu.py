@@ -134,9 +134,10 @@ def test_decode_append_rejections(lib):
 def test_attention_backward_rejections(lib):
     fn = lib.ssa_sparse_attn_bwd
     names = ["Q", "K", "V", "O", "dO", "lse", "dt", "idx", "cnt", "batch", "Hq", "Hkv", "N", "d",
-             "B", "max_sel", "scale", "dQ", "dK", "dV", "delta", "stream"]
+             "B", "max_sel", "scale", "dQ", "dK", "dV", "ws", "ws_bytes", "stream"]
+    need = abi.ssa_sparse_attn_bwd_workspace_size(1, 8, 2, 4096, 128, 64)
     ok = [FAKE] * 6 + [1, FAKE, FAKE, 1, 8, 2, 4096, 128, 64, 18, 0.088, FAKE, FAKE, FAKE, FAKE,
-                       NULL]
+                       need, NULL]
 
     def call(**kw):
         args = list(ok)
@@ -152,9 +153,13 @@ def test_attention_backward_rejections(lib):
     assert call(N=0) == 1
     assert call(max_sel=0) == 1
     assert call(scale=0.0) == 1
-    for name in ("Q", "K", "V", "O", "dO", "lse", "idx", "cnt", "dQ", "dK", "dV", "delta"):
+    for name in ("Q", "K", "V", "O", "dO", "lse", "idx", "cnt", "dQ", "dK", "dV", "ws"):
         assert call(**{name: NULL}) == 1, name
     assert call(dK=ctypes.c_void_p(0x100008)) == 1  # not 16-byte aligned
+    assert call(ws=ctypes.c_void_p(0x100010)) == 1  # workspace not 256-byte aligned
+    assert call(ws_bytes=need - 1) == 1             # workspace too small
+    # delta for every query row, then the sink block's partial sums
+    assert need >= 1 * 8 * 4096 * 4 + 1 * 2 * 2 * 64 * 128 * 4
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

@@ -73,6 +73,8 @@ def _check(gpu, ref):
     (2, 8, 2, 128 * 5 + 40, 128, 128, 2, 3),    # B = 128 (8 warps), ragged, batch 2
     (1, 2, 2, 16 * 40, 64, 16, 4, 5),           # B = 16: one warp, a chunk wider than B
     (1, 4, 4, 64 * 300, 128, 64, 4, 8),         # > 128 query blocks per key-block scan
+    (1, 8, 2, 64 * 150 + 5, 128, 64, 4, 5),     # GQA 4: the sink column in 3 ranges of 64
+    (2, 4, 2, 128 * 70, 64, 128, 3, 4),         # B = 128, sink in 3 ranges of 32, batch 2
 ])
 def test_backward_parity(ssa, batch, Hq, Hkv, N, d, B, topk, clusters):
     gpu, ref, _ = _case(ssa, batch, Hq, Hkv, N, d, B, topk, clusters, seed=21)
@@ -113,7 +115,8 @@ def test_backward_zero_outside_every_selection(ssa):
 
 
 def test_backward_is_deterministic(ssa):
-    batch, Hq, Hkv, N, d, B, topk = 1, 8, 2, 64 * 40, 128, 64, 6
+    # 150 query blocks: the sink block's dK / dV are summed over three ranges
+    batch, Hq, Hkv, N, d, B, topk = 1, 8, 2, 64 * 150, 128, 64, 6
     Q, K, V = planted_prefill(batch, Hq, Hkv, N, d, B, 6, seed=25, dtype="bf16", device=DEV)
     dO = upstream_grad(batch, Hq, N, d, seed=26, dtype="bf16", device=DEV)
     idx, cnt = ssa.ssa_route(Q, ssa.ssa_block_summary(K, B), B, topk, Hkv)
