@@ -382,7 +382,8 @@ ssa_status ssa_device_error(int* code) {
   if (cudaDeviceSynchronize() != cudaSuccess) return SSA_ERR_CUDA;
   int a = ssa::read_and_reset_attn_tc_error();
   int b = ssa::read_and_reset_decode_error();
-  *code = a != 0 ? a : b;
+  int c = ssa::read_and_reset_bwd_tc_error();
+  *code = a != 0 ? a : (b != 0 ? b : c);
   return SSA_OK;
 }
 
@@ -391,7 +392,8 @@ ssa_status ssa_check_device_error(ssa_stream stream, int* code) {
   ErrorWords words{};
   if (ssa::attn_tc_error_word(&words.w[0]) != cudaSuccess) return SSA_ERR_CUDA;
   if (ssa::decode_error_word(&words.w[1]) != cudaSuccess) return SSA_ERR_CUDA;
-  words.n = 2;
+  if (ssa::bwd_tc_error_word(&words.w[2]) != cudaSuccess) return SSA_ERR_CUDA;
+  words.n = 3;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   take_error_words_kernel<<<1, 1, 0, s>>>(words);
   if (cudaGetLastError() != cudaSuccess) return SSA_ERR_CUDA;

@@ -603,22 +603,33 @@ static cudaError_t launch_bwd_t(const BwdPlan& pl, const void* Q, const void* K,
                                                                    delta, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+  const bool tc = attn_tc_supported(SSA_BF16, Hq, Hkv, D, B);
+  if (tc) {
+    e = launch_bwd_dq_tc(Q, K, V, dO, lse, delta, idx, cnt, batch, Hq, Hkv, N, B, max_sel, scale,
+                         dQ, st);
+  } else {
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_dq_kernel<D><<<(unsigned)((long long)batch * Hq * nq), threads, smem, st>>>(
+        (const bf*)Q, (const bf*)K, (const bf*)V, (const bf*)dO, lse, delta, idx, cnt, Hq, Hkv,
+        N, B, nq, max_sel, scale, (bf*)dQ);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<(unsigned)((long long)batch * Hq * nq), threads, smem, st>>>(
-      (const bf*)Q, (const bf*)K, (const bf*)V, (const bf*)dO, lse, delta, idx, cnt, Hq, Hkv, N,
-      B, nq, max_sel, scale, (bf*)dQ);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-  if (e != cudaSuccess) return e;
-  const long long ctas = (long long)nbg * pl.sink_nsplit + (long long)nbg * (nq - 1);
-  bwd_dkv_kernel<D><<<(unsigned)ctas, threads, smem, st>>>(
-      (const bf*)Q, (const bf*)K, (const bf*)V, (const bf*)dO, lse, delta, idx, cnt, batch, Hq,
-      Hkv, N, B, nq, max_sel, scale, (bf*)dK, (bf*)dV, part, pl.sink_qr, pl.sink_nsplit);
-  e = cudaGetLastError();
+  if (tc && B == 64) {
+    e = launch_bwd_dkv_tc(Q, K, V, dO, lse, delta, idx, cnt, batch, Hq, Hkv, N, max_sel, scale,
+                          dK, dV, part, pl.sink_qr, pl.sink_nsplit, st);
+  } else {
+    e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long ctas = (long long)nbg * pl.sink_nsplit + (long long)nbg * (nq - 1);
+    bwd_dkv_kernel<D><<<(unsigned)ctas, threads, smem, st>>>(
+        (const bf*)Q, (const bf*)K, (const bf*)V, (const bf*)dO, lse, delta, idx, cnt, batch, Hq,
+        Hkv, N, B, nq, max_sel, scale, (bf*)dK, (bf*)dV, part, pl.sink_qr, pl.sink_nsplit);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   const dim3 rgrid((unsigned)((B * D + 255) / 256), (unsigned)nbg);
   bwd_sink_reduce_kernel<D><<<rgrid, 256, 0, st>>>(part, nbg, pl.sink_nsplit, B, N, scale,

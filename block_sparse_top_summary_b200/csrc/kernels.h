@@ -50,6 +50,18 @@ struct BwdPlan {
 };
 BwdPlan plan_bwd(int batch, int Hq, int Hkv, int N, int d, int B);
 size_t attn_bwd_smem_bytes(int d, int B);
+// Tensor-core (tcgen05) forms of the two contraction passes, for the shapes of
+// attn_tc_supported (dK / dV: B = 64 only); the sink ranges as in the
+// mma.sync form.
+cudaError_t launch_bwd_dq_tc(const void* Q, const void* K, const void* V, const void* dO,
+                             const float* lse, const float* delta, const int32_t* idx,
+                             const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
+                             int max_sel, float scale, void* dQ, cudaStream_t st);
+cudaError_t launch_bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO,
+                              const float* lse, const float* delta, const int32_t* idx,
+                              const int32_t* cnt, int batch, int Hq, int Hkv, int N,
+                              int max_sel, float scale, void* dK, void* dV, float* sink_part,
+                              int sink_qr, int sink_nsplit, cudaStream_t st);
 cudaError_t launch_attn_bwd(const BwdPlan& pl, const void* Q, const void* K, const void* V,
                             const void* O, const void* dO, const float* lse, const int32_t* idx,
                             const int32_t* cnt, int batch, int Hq, int Hkv, int N, int d, int B,
@@ -103,5 +115,7 @@ int read_and_reset_decode_error();
 // Device addresses of the same words (current device), for stream-ordered reads.
 cudaError_t attn_tc_error_word(int** word);
 cudaError_t decode_error_word(int** word);
+int read_and_reset_bwd_tc_error();
+cudaError_t bwd_tc_error_word(int** word);
 
 }  // namespace ssa

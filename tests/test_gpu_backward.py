@@ -75,6 +75,10 @@ def _check(gpu, ref):
     (1, 4, 4, 64 * 300, 128, 64, 4, 8),         # > 128 query blocks per key-block scan
     (1, 8, 2, 64 * 150 + 5, 128, 64, 4, 5),     # GQA 4: the sink column in 3 ranges of 64
     (2, 4, 2, 128 * 70, 64, 128, 3, 4),         # B = 128, sink in 3 ranges of 32, batch 2
+    # tensor-core passes (bf16, d = 128, G * B a multiple of 256):
+    (1, 8, 2, 64 * 20 + 7, 128, 64, 4, 3),      # dQ and dK/dV on tcgen05, ragged tail
+    (2, 16, 4, 64 * 33, 128, 64, 6, 5),         # the same, batch 2, GQA 4
+    (1, 4, 2, 128 * 9 + 5, 128, 128, 3, 3),     # dQ on tcgen05 at B = 128, GQA 2
 ])
 def test_backward_parity(ssa, batch, Hq, Hkv, N, d, B, topk, clusters):
     gpu, ref, _ = _case(ssa, batch, Hq, Hkv, N, d, B, topk, clusters, seed=21)
@@ -87,10 +91,11 @@ def test_backward_all_blocks_selected(ssa):
     _check(gpu, ref)
 
 
-def test_backward_zero_outside_every_selection(ssa):
+@pytest.mark.parametrize("Hq", [4, 8])  # 8: the tensor-core passes
+def test_backward_zero_outside_every_selection(ssa, Hq):
     # dO nonzero on one query block only: dK and dV are exactly zero on every
     # key that block does not attend
-    batch, Hq, Hkv, N, d, B, topk = 1, 4, 2, 64 * 12, 128, 64, 2
+    batch, Hkv, N, d, B, topk = 1, 2, 64 * 12, 128, 64, 2
     Q, K, V = planted_prefill(batch, Hq, Hkv, N, d, B, 4, seed=23, dtype="bf16")
     dO = upstream_grad(batch, Hq, N, d, seed=24, dtype="bf16")
     i = 9
