@@ -9,7 +9,8 @@
 // rows).  The selected blocks are visited in chunks of 128 keys (two blocks at
 // B = 64, one at B = 128; an odd last block is paired with an all-zero
 // out-of-range box whose keys are masked).  One persistent CTA per SM runs a
-// sequence of work items back to back.
+// sequence of work items back to back, the heaviest first within each group
+// of (batch, KV head) pairs.
 //
 // Roles (576 threads, 18 warps):
 //   warp 0      TMA producer: Q of each work item (8 boxes of 64 x 64 bf16,
@@ -218,18 +219,26 @@ __device__ __forceinline__ void exp_pack32(const uint32_t (&v)[32], uint32_t (&w
 
 }  // namespace
 
-// Work item w (heaviest first: query block i = nq - 1 - w / (subs * nbg)).
+// Work item w.  The (batch, KV head) pairs are taken in groups of `kvg`
+// (the last group may be smaller); within a group, the heaviest query blocks
+// (the latest) come first.  A group's K and V are what the CTAs read at one
+// time, so the host sizes it to stay near the L2.
 struct Item {
   int b, g, i, h0, bg;
 };
 
-__device__ __forceinline__ Item item_of(int w, int subs, int nbg, int Hkv, int G, int nq, int HPI) {
+__device__ __forceinline__ Item item_of(int w, int subs, int nbg, int Hkv, int G, int nq, int HPI,
+                                        int kvg) {
   Item it;
-  const int per_i = subs * nbg;
-  it.i = nq - 1 - w / per_i;
-  const int rem = w - (w / per_i) * per_i;
-  it.bg = rem / subs;
-  const int sub = rem - it.bg * subs;
+  const int per_grp = kvg * subs * nq;
+  const int grp = w / per_grp;
+  const int rem = w - grp * per_grp;
+  const int gn = min(kvg, nbg - grp * kvg);  // pairs in this group
+  const int per_i = gn * subs;
+  it.i = nq - 1 - rem / per_i;
+  const int rem2 = rem - (rem / per_i) * per_i;
+  it.bg = grp * kvg + rem2 / subs;
+  const int sub = rem2 - (rem2 / subs) * subs;
   it.b = it.bg / Hkv;
   it.g = it.bg - it.b * Hkv;
   it.h0 = it.g * G + sub * HPI;
@@ -252,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
-    int Hq, int Hkv, int N, int nq, int nbg, int max_sel, float scale_log2) {
+    int Hq, int Hkv, int N, int nq, int nbg, int max_sel, float scale_log2, int kvg) {
   constexpr int HPT = 128 / B;      // query heads per M-tile
   constexpr int HPI = 2 * HPT;      // query heads per work item
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -271,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   volatile int* abort = &sh->abort;
   auto ns_of = [&](int w) -> int {
     if (w >= W) return 0;
-    const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI);
+    const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI, kvg);
     return cnt[(int64_t)it.bg * nq + it.i];
   };
 
@@ -314,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     int gc = 0, kq = 0;
     bool ok = true;
     for (int w = blockIdx.x; ok && w < W; w += gridDim.x) {
-      const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI);
+      const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI, kvg);
       const int ns = cnt[(int64_t)it.bg * nq + it.i];
       const int nch = chunks_of<B>(ns);
       if (nch == 0) continue;
@@ -466,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       ns_next = ns_of(w + gridDim.x);
       const int nch = chunks_of<B>(ns);
       if (nch == 0) continue;
-      const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI);
+      const Item it = item_of(w, subs, nbg, Hkv, G, nq, HPI, kvg);
       const int hh = r / B;
       const int pos = it.i * B + (r % B);
       const int h = it.h0 + t * HPT + hh;
@@ -681,9 +690,14 @@ cudaError_t launch_tc_t(const void* Q, const void* K, const void* V, const int32
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int grid = (int)(items < sms ? items : sms);  // one persistent CTA per SM
+  // (batch, KV head) pairs per group of items: all of them while their K and
+  // V fit in twice the L2 (126 MB), else two at a time
+  const int nbg = batch * Hkv;
+  const double kv_bytes = 2.0 * N * 128 * 2;  // K and V of one pair
+  const int kvg = (nbg * kv_bytes <= 2.0 * 126e6) ? nbg : (nbg < 2 ? nbg : 2);
   attn_tc_kernel<B><<<grid, kThreads, smem, st>>>(mq, mk, mv, idx, cnt, (__nv_bfloat16*)O, lse,
-                                                  Hq, Hkv, N, nq, batch * Hkv, max_sel,
-                                                  scale * 1.4426950408889634f);
+                                                  Hq, Hkv, N, nq, nbg, max_sel,
+                                                  scale * 1.4426950408889634f, kvg);
   return cudaGetLastError();
 }
 
