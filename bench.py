@@ -28,7 +28,12 @@ Timed apart from the step and reported under their own keys:
   calls, every append completing a block);
 - `kernels.ssa_sparse_attn_bwd`: the backward of the 32K prefill attention on
   its own selection (8 * d FLOPs per unmasked pair: the dV, dP, dQ and dK
-  contractions).
+  contractions);
+- `widened`: the calls beyond the four steps -- decode over a paged copy of the
+  decode cache (checked bitwise against the contiguous decode) and with one
+  selection per query head, two-level routing on the 128K prefill, and
+  DashAttention's learned summary, alpha-entmax routing and prior attention
+  on the 32K prefill -- each with its bytes or FLOPs and fraction of peak.
 Every kernel line carries its fraction of the measured peak (MEASURED_PEAKS)
 and of the nominal one (2.25 PFLOP/s dense bf16, 8 TB/s HBM).
 
@@ -81,6 +86,27 @@ def decode_bytes(idx: np.ndarray, seqlens: np.ndarray, B: int, d: int, G: int, e
             total += 2.0 * rows * d * esize
             total += max(last - 1, 0) * d * 4.0
     total += 2.0 * batch * Hkv * G * d * esize
+    return total
+
+
+def per_head_decode_bytes(idx: np.ndarray, seqlens: np.ndarray, B: int, d: int, G: int,
+                          esize: int) -> float:
+    """The bytes decode with one selection per query head (idx ``[batch, Hq, w]``)
+    must move: the K and V rows of the union of the selections of a KV head's G
+    query heads (a block two heads select is read once), the KV head's candidate
+    summaries once, and every head's q and O rows."""
+    total = 0.0
+    batch, Hq, _ = idx.shape
+    Hkv = Hq // G
+    for b in range(batch):
+        L = int(seqlens[b])
+        last = (L - 1) // B
+        for g in range(Hkv):
+            grp = idx[b, g * G:(g + 1) * G]
+            sel = np.unique(grp[grp >= 0])
+            rows = np.minimum(B, L - sel * B).sum()
+            total += 2.0 * rows * d * esize + max(last - 1, 0) * d * 4.0
+    total += 2.0 * batch * Hq * d * esize
     return total
 
 
@@ -322,6 +348,105 @@ def prefill_report(p: Prefill, seg, flops, hbm_peak, bf16_peak, tc):
     }
 
 
+def time_call(f, iters: int, warmup: int, stream, world) -> float:
+    """Mean device time (ms) of f() over `iters` calls after `warmup` calls."""
+    for _ in range(warmup):
+        f()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b_ = _ev(), _ev()
+    a.record(stream)
+    for _ in range(iters):
+        f()
+    b_.record(stream)
+    torch.cuda.synchronize()
+    return max_over_ranks(a.elapsed_time(b_) / iters, world)
+
+
+def widened(ssa, p128, p32, q, Kc, Vc, Sc, L, cd, dev, stream, world, hbm_peak, bf16_peak):
+    """The rows beyond the four hot-path steps, each on a workload of the
+    benchmark, with its own work count and fraction of peak."""
+    out = {}
+
+    def hbm(ms, nbytes, workload, **kw):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "GB/s": gbs, **fracs(gbs, hbm_peak, NOMINAL_HBM_GBS), "bytes": nbytes,
+                "workload": workload, **kw}
+
+    # paged decode: the decode workload's cache cut into pages in a shuffled order
+    nblk = cd.L // cd.B
+    gen = torch.Generator(device=dev).manual_seed(7)
+    perm = torch.randperm(cd.batch * nblk, generator=gen, device=dev)
+    Kp = torch.empty(cd.batch * nblk, cd.Hkv, cd.B, cd.d, dtype=Kc.dtype, device=dev)
+    Vp = torch.empty_like(Kp)
+    Kp[perm] = Kc.view(cd.batch, cd.Hkv, nblk, cd.B, cd.d).transpose(1, 2).reshape(-1, cd.Hkv, cd.B, cd.d)
+    Vp[perm] = Vc.view(cd.batch, cd.Hkv, nblk, cd.B, cd.d).transpose(1, 2).reshape(-1, cd.Hkv, cd.B, cd.d)
+    table = perm.view(cd.batch, nblk).to(torch.int32).contiguous()
+    ws = torch.empty(ssa.ssa_decode_workspace_size(cd.batch, cd.Hq, cd.Hkv, cd.L, cd.d, cd.B,
+                                                   cd.topk), dtype=torch.uint8, device=dev)
+    Op = torch.empty_like(q)
+    ip = torch.empty(cd.batch, cd.Hkv, ssa.decode_width(cd.L, cd.B, cd.topk), dtype=torch.int32,
+                     device=dev)
+    f = lambda: ssa.ssa_decode_paged(q, Kp, Vp, Sc, table, L, cd.B, cd.topk, O=Op, idx=ip,
+                                     workspace=ws)
+    ms = time_call(f, 20, 3, stream, world)
+    Oc, ic = ssa.ssa_decode(q, Kc, Vc, Sc, L, cd.B, cd.topk)
+    assert torch.equal(Op, Oc) and torch.equal(ip, ic), "paged decode differs from the contiguous one"
+    nb = decode_bytes(ip.cpu().numpy(), L.cpu().numpy(), cd.B, cd.d, cd.Hq // cd.Hkv, 2)
+    out["ssa_decode_paged"] = hbm(ms, nb, "decode (64 seq x 65536) in 65536 pages, shuffled",
+                                  tokens_per_s=cd.batch / (ms * 1e-3))
+    del Kp, Vp
+    # per-head decode routing on the decode workload
+    wsh = torch.empty(ssa.ssa_decode_per_head_workspace_size(cd.batch, cd.Hq, cd.Hkv, cd.L, cd.d,
+                                                             cd.B, cd.topk),
+                      dtype=torch.uint8, device=dev)
+    Oh = torch.empty_like(q)
+    ih = torch.empty(cd.batch, cd.Hq, ssa.decode_width(cd.L, cd.B, cd.topk), dtype=torch.int32,
+                     device=dev)
+    f = lambda: ssa.ssa_decode_per_head(q, Kc, Vc, Sc, L, cd.B, cd.topk, O=Oh, idx=ih,
+                                        workspace=wsh)
+    ms = time_call(f, 20, 3, stream, world)
+    nb = per_head_decode_bytes(ih.cpu().numpy(), L.cpu().numpy(), cd.B, cd.d, cd.Hq // cd.Hkv, 2)
+    out["ssa_decode_per_head"] = hbm(ms, nb, "decode (64 seq x 65536), one selection per query head",
+                                     tokens_per_s=cd.batch / (ms * 1e-3))
+    # two-level routing on the 128K prefill: segments of 8 blocks, 8 kept, 32 blocks
+    c = p128.c
+    hi = torch.empty(c.batch, c.Hkv, -(-c.N // c.B), min(c.topk, -(-c.N // c.B)) + 2,
+                     dtype=torch.int32, device=dev)
+    hc = torch.empty(c.batch, c.Hkv, -(-c.N // c.B), dtype=torch.int32, device=dev)
+    f = lambda: ssa.ssa_route_hierarchical(p128.Q, p128.S, c.B, 8, 8, c.topk, c.Hkv, idx=hi,
+                                           cnt=hc)
+    ms = time_call(f, 10, 3, stream, world)
+    out["ssa_route_hierarchical"] = hbm(ms, p128.route_bytes(),
+                                        describe(c) + ", segments of 8 blocks, 8 kept")
+    # DashAttention's stages on the 32K prefill
+    c = p32.c
+    qbar = torch.randn(c.Hkv, c.d, generator=gen, device=dev)
+    S_l = torch.empty_like(p32.S)
+    f = lambda: ssa.ssa_learned_summary(p32.K, qbar, c.B, S=S_l)
+    ms = time_call(f, 20, 3, stream, world)
+    out["ssa_learned_summary"] = hbm(ms, p32.summary_bytes(), describe(c))
+    f = lambda: ssa.ssa_route_entmax(p32.Q, p32.S, c.B, c.Hkv, 1.5, 8.0, 0.5)
+    ms = time_call(f, 10, 3, stream, world)
+    ei, ec, eb, _ = ssa.ssa_route_entmax(p32.Q, p32.S, c.B, c.Hkv, 1.5, 8.0, 0.5)
+    nb = p32.Q.numel() * 2 + p32.S.numel() * 4 + ei.numel() * 8 + ec.numel() * 4
+    out["ssa_route_entmax"] = hbm(ms, nb, describe(c) + ", alpha 1.5, gamma 8, sigma 0.5",
+                                  mean_blocks=float(ec.float().mean()))
+    Oe = torch.empty_like(p32.Q)
+    f = lambda: ssa.ssa_sparse_attn_fwd_prior(p32.Q, p32.K, p32.V, ei, ec, eb, c.B, O=Oe)
+    ms = time_call(f, 3, 1, stream, world)
+    ecn = ec.cpu().numpy()
+    fl = sum(attn_flops(ecn[b, g], c.N, c.B, c.Hq // c.Hkv, c.d)
+             for b in range(c.batch) for g in range(c.Hkv))
+    tf = fl / (ms * 1e-3) / 1e12
+    out["ssa_sparse_attn_fwd_prior"] = {"ms": ms, "TFLOP/s": tf, "bound": "alu",
+                                        "flops": fl, "workload": describe(c) + ", entmax selection",
+                                        "note": "CUDA cores (FFMA); fraction of the bf16 tensor "
+                                                "peak given for scale only",
+                                        **fracs(tf, bf16_peak, NOMINAL_BF16_TFLOPS)}
+    return out
+
+
 def run_ours(args, world, rank, local):
     import block_sparse_top_summary_b200 as ssa
     ssa.load_library()
@@ -429,8 +554,6 @@ def run_ours(args, world, rank, local):
                                ssa.ssa_sparse_attn_uses_tensor_cores(
                                    torch.bfloat16, po.c.Hq, po.c.Hkv, po.c.d, po.c.B))
     p32 = P if head == "prefill32k" else po  # the backward runs on the 32K workload
-    if head == "prefill32k":
-        del po
 
     # --- the sparsity sweep: attention TFLOP/s against k, "all" last
     cs = CONFIGS["sweep"]
@@ -514,6 +637,9 @@ def run_ours(args, world, rank, local):
     # 8 d per unmasked (query, key) pair: the dV, dP, dQ and dK contractions
     bwd_flops = 2.0 * p32.flops()
     bwd_tflops = bwd_flops / (bwd_ms * 1e-3) / 1e12
+    del dQb, dKb, dVb, bws
+    wide = widened(ssa, P if head == "prefill128k" else po, p32, q, Kc, Vc, Sc, L, cd, dev, stream,
+                   world, hbm_peak, bf16_peak)
     assert ssa.ssa_device_error() == 0
 
     kernels = {k: head_rep[k] for k in ("ssa_block_summary", "ssa_route", "ssa_sparse_attn_fwd")}
@@ -557,6 +683,7 @@ def run_ours(args, world, rank, local):
         other: other_rep,
         "sweep": {"workload": describe(cs, "k"),
                   "points": sweep},
+        "widened": wide,
         "e2e": {"value": all_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * 5,

@@ -47,3 +47,33 @@ def test_decode_bytes_counts_the_rows_each_selection_reads():
             expect += 2 * rows * d * esize + len(range(1, max(last, 1))) * d * 4
     expect += 2 * batch * Hq * d * esize
     assert bench.decode_bytes(idx, L, B, d, Hq // Hkv, esize) == expect
+
+
+def test_per_head_decode_bytes_counts_the_union_of_a_groups_rows():
+    # the K/V rows of the blocks any head of a KV head's group selects (once),
+    # that KV head's candidate summaries (once), and every head's q and O
+    rng = np.random.default_rng(6)
+    batch, Hq, Hkv, Lmax, d, B, topk = 2, 4, 2, 8 * 9, 8, 8, 2
+    G = Hq // Hkv
+    L = np.array([72, 30])
+    idx = np.full((batch, Hq, topk + 2), -1)
+    for b in range(batch):
+        last = (L[b] - 1) // B
+        for h in range(Hq):
+            cand = rng.choice(np.arange(1, max(last, 2)), size=min(topk, max(last - 1, 0)),
+                              replace=False) if last > 1 else np.array([], dtype=int)
+            sel = sorted({0, last} | set(int(c) for c in cand))
+            idx[b, h, :len(sel)] = sel
+    esize = 2
+    expect = 0.0
+    for b in range(batch):
+        last = (L[b] - 1) // B
+        for g in range(Hkv):
+            sel = set(int(j) for h in range(g * G, (g + 1) * G) for j in idx[b, h] if j >= 0)
+            rows = sum(1 for t in range(L[b]) if t // B in sel)
+            expect += 2 * rows * d * esize + len(range(1, max(last, 1))) * d * 4
+    expect += 2 * batch * Hq * d * esize
+    assert bench.per_head_decode_bytes(idx, L, B, d, G, esize) == expect
+    # one head per group: the grouped count
+    assert bench.per_head_decode_bytes(idx[:, ::2], L, B, d, 1, esize) == \
+        bench.decode_bytes(idx[:, ::2], L, B, d, 1, esize)
