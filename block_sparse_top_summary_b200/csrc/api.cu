@@ -107,7 +107,8 @@ ssa_status ssa_sparse_attn_fwd(const void* Q, const void* K, const void* V, ssa_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (ssa::attn_tc_supported(dtype, Hq, Hkv, d, B))
     return from_cuda(
-        ssa::launch_attn_tc(Q, K, V, idx, cnt, batch, Hq, Hkv, N, B, max_sel, scale, O, lse, s));
+        ssa::launch_attn_tc(Q, K, V, idx, cnt, nullptr, batch, Hq, Hkv, N, B, max_sel, scale, O,
+                            lse, s));
   return from_cuda(ssa::launch_attn_simt(Q, K, V, dtype, idx, cnt, nullptr, batch, Hq, Hkv, N, d,
                                          B, max_sel, scale, O, lse, s));
 }
@@ -160,9 +161,12 @@ ssa_status ssa_sparse_attn_fwd_prior(const void* Q, const void* K, const void* V
     return SSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return SSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (ssa::attn_tc_supported(dtype, Hq, Hkv, d, B))
+    return from_cuda(ssa::launch_attn_tc(Q, K, V, idx, cnt, bias, batch, Hq, Hkv, N, B, max_sel,
+                                         scale, O, lse, s));
   return from_cuda(ssa::launch_attn_simt(Q, K, V, dtype, idx, cnt, bias, batch, Hq, Hkv, N, d, B,
-                                         max_sel, scale, O, lse,
-                                         reinterpret_cast<cudaStream_t>(stream)));
+                                         max_sel, scale, O, lse, s));
 }
 
 ssa_status ssa_sparse_attn_bwd_workspace_size(int batch, int Hq, int Hkv, int N, int d, int B,

@@ -29,6 +29,8 @@
 //               exceeds it by more than 2^64),
 //               write P as bf16 pairs into the first 32 columns of the thread's
 //               own S half (tcgen05.st), and finally normalise O and store it.
+//               With a routing prior (DashAttention's stage 2) each half's
+//               block adds its offset to the scaled logits.
 // TMEM columns: S of tile t at 128 t (P of keys 0-63 at 128 t, of keys 64-127
 // at 128 t + 64), O of tile t at 256 + 128 t.
 // Every mbarrier wait is bounded in time; on expiry the CTA records
@@ -256,11 +258,16 @@ __device__ __forceinline__ int chunks_of(int ns) {
 // once the last S of the current one completes, its first S runs while the
 // current item's epilogue reads O, and its first P.V waits only for that
 // epilogue (o_free).
-template <int B>
+// PRIOR: the kernel adds a routing prior per selected block (the bias
+// argument); the plain kernel is compiled without that code.  At most 96
+// registers per thread: the 18 warps of a CTA share four register quarters of
+// the SM, one of which holds 5 of them (5 x 32 x 96 fits 16K).
+template <int B, bool PRIOR>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ idx,
-    const int32_t* __restrict__ cnt, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
+    const int32_t* __restrict__ cnt, const float* __restrict__ bias,
+    __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
     int Hq, int Hkv, int N, int nq, int nbg, int max_sel, float scale_log2, int kvg) {
   constexpr int HPT = 128 / B;      // query heads per M-tile
   constexpr int HPI = 2 * HPT;      // query heads per work item
@@ -479,9 +486,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       const int hh = r / B;
       const int pos = it.i * B + (r % B);
       const int h = it.h0 + t * HPT + hh;
+      // the routing prior of each selected block (natural log)
+      const float* brow = PRIOR ? bias + ((int64_t)it.bg * nq + it.i) * max_sel : nullptr;
       float m_used = -INFINITY, l = 0.f;
       for (int c = 0; c < nch; ++c) {
         const int g = gc + c;
+        // this half's block: entry 2c + half (B = 64) or c (B = 128); its
+        // prior joins the logits in the log2 domain
+        const int ent = (B == 64) ? 2 * c + half : c;
+        const float bh = (PRIOR && ent < ns) ? brow[ent] * 1.4426950408889634f : 0.f;
         if (!(ok = warp_wait_bar(&sh->s_full[t], g & 1, abort))) break;
         ptx::tc_fence_after();
         const bool last = (c == nch - 1);
@@ -515,7 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           if (last) mask32<B>(v, half * 64 + q * 32, lim);
           pm = max32(v, pm);
         }
-        sh->mx[g & 1][t][half][r] = pm;
+        // the half's max of the scaled logits (with the prior), exchanged
+        const float pmb = PRIOR ? pm * scale_log2 + bh : pm * scale_log2;
+        sh->mx[g & 1][t][half][r] = pmb;
         ptx::mbar_arrive(&sh->mx_full[t]);
         // The two halves of a row must use one reference max.  From chunk 1
         // on, P is computed optimistically with the current reference m_used
@@ -528,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         bool have_rmax = false;
         if (c == 0) {
           if (!(ok = warp_wait_bar(&sh->mx_full[t], g & 1, abort))) break;
-          rmax = fmaxf(pm, sh->mx[g & 1][t][half ^ 1][r]) * scale_log2;
+          rmax = fmaxf(pmb, sh->mx[g & 1][t][half ^ 1][r]);
           m_used = rmax;
           have_rmax = true;
         }
@@ -539,7 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         for (int attempt = 0; attempt < 2; ++attempt) {
           const float mu = (m_used == -INFINITY) ? 0.f : m_used;
           const uint64_t s2 = pack2(scale_log2, scale_log2);
-          const uint64_t c2 = pack2(-mu, -mu);
+          const float cst = PRIOR ? bh - mu : -mu;
+          const uint64_t c2 = pack2(cst, cst);
           // pass 2: p = 2^(s*scale - m) as bf16 pairs (S stays intact until
           // the pairs are stored, so a redo can read it again)
           acc = 0;
@@ -556,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           }
           if (!have_rmax) {
             if (!(ok = warp_wait_bar(&sh->mx_full[t], g & 1, abort))) break;
-            rmax = fmaxf(pm, sh->mx[g & 1][t][half ^ 1][r]) * scale_log2;
+            rmax = fmaxf(pmb, sh->mx[g & 1][t][half ^ 1][r]);
             have_rmax = true;
           }
           // both halves of a row see the same rmax and m_used, so they decide
@@ -669,8 +685,8 @@ namespace {
 
 template <int B>
 cudaError_t launch_tc_t(const void* Q, const void* K, const void* V, const int32_t* idx,
-                        const int32_t* cnt, int batch, int Hq, int Hkv, int N, int max_sel,
-                        float scale, void* O, float* lse, cudaStream_t st) {
+                        const int32_t* cnt, const float* bias, int batch, int Hq, int Hkv, int N,
+                        int max_sel, float scale, void* O, float* lse, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
   if (!make_bf16_map(&mq, Q, 128, N, batch * Hq, 64) ||
       !make_bf16_map(&mk, K, 128, N, batch * Hkv, 64) ||
@@ -683,7 +699,8 @@ cudaError_t launch_tc_t(const void* Q, const void* K, const void* V, const int32
   if (items <= 0) return cudaSuccess;
   if (items > (1ll << 30)) return cudaErrorInvalidValue;
   const size_t smem = 1024 + kSmemBytes + sizeof(Shared);
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = bias != nullptr ? attn_tc_kernel<B, true> : attn_tc_kernel<B, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
@@ -695,7 +712,7 @@ cudaError_t launch_tc_t(const void* Q, const void* K, const void* V, const int32
   const int nbg = batch * Hkv;
   const double kv_bytes = 2.0 * N * 128 * 2;  // K and V of one pair
   const int kvg = (nbg * kv_bytes <= 2.0 * 126e6) ? nbg : (nbg < 2 ? nbg : 2);
-  attn_tc_kernel<B><<<grid, kThreads, smem, st>>>(mq, mk, mv, idx, cnt, (__nv_bfloat16*)O, lse,
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, idx, cnt, bias, (__nv_bfloat16*)O, lse,
                                                   Hq, Hkv, N, nq, nbg, max_sel,
                                                   scale * 1.4426950408889634f, kvg);
   return cudaGetLastError();
@@ -710,13 +727,14 @@ bool attn_tc_supported(ssa_dtype dt, int Hq, int Hkv, int d, int B) {
 }
 
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const int32_t* idx,
-                           const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
-                           int max_sel, float scale, void* O, float* lse, cudaStream_t st) {
+                           const int32_t* cnt, const float* bias, int batch, int Hq, int Hkv,
+                           int N, int B, int max_sel, float scale, void* O, float* lse,
+                           cudaStream_t st) {
   if (max_sel > 8192) return cudaErrorInvalidValue;
-  return B == 64 ? launch_tc_t<64>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, max_sel, scale, O, lse,
-                                   st)
-                 : launch_tc_t<128>(Q, K, V, idx, cnt, batch, Hq, Hkv, N, max_sel, scale, O, lse,
-                                    st);
+  return B == 64 ? launch_tc_t<64>(Q, K, V, idx, cnt, bias, batch, Hq, Hkv, N, max_sel, scale, O,
+                                   lse, st)
+                 : launch_tc_t<128>(Q, K, V, idx, cnt, bias, batch, Hq, Hkv, N, max_sel, scale, O,
+                                    lse, st);
 }
 
 cudaError_t attn_tc_error_word(int** word) {

@@ -23,9 +23,12 @@ cudaError_t launch_route(const void* Q, ssa_dtype dt, const float* S, int batch,
 // True when the tensor-core prefill kernel covers this shape.
 bool attn_tc_supported(ssa_dtype dt, int Hq, int Hkv, int d, int B);
 
+// bias: NULL, or the routing prior of each selection entry (natural log) added
+// to the scaled logits of that block's keys.
 cudaError_t launch_attn_tc(const void* Q, const void* K, const void* V, const int32_t* idx,
-                           const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
-                           int max_sel, float scale, void* O, float* lse, cudaStream_t st);
+                           const int32_t* cnt, const float* bias, int batch, int Hq, int Hkv,
+                           int N, int B, int max_sel, float scale, void* O, float* lse,
+                           cudaStream_t st);
 
 cudaError_t launch_attn_simt(const void* Q, const void* K, const void* V, ssa_dtype dt,
                              const int32_t* idx, const int32_t* cnt, const float* bias, int batch,

@@ -187,7 +187,10 @@ ssa_status ssa_route_entmax(const void* Q, ssa_dtype dtype, const float* S, int 
  * on the diagonal):
  *   O[b, h, t] = softmax(scale * q_t . K_sel^T + bias_sel) V_sel.
  * idx, cnt, bias as written by ssa_route_entmax (bias [batch, Hkv, nq,
- * max_sel] fp32).  Runs on the CUDA cores (FFMA online softmax).
+ * max_sel] fp32).  The shapes of ssa_sparse_attn_fwd's tensor-core path (bf16,
+ * d = 128, B in {64, 128}, (Hq/Hkv)*B a multiple of 256) run on that kernel,
+ * with the offset joining each block's scaled logits; others run the FFMA
+ * kernel.
  */
 ssa_status ssa_sparse_attn_fwd_prior(const void* Q, const void* K, const void* V,
                                      ssa_dtype dtype, const int32_t* idx, const int32_t* cnt,

@@ -96,11 +96,14 @@ def test_entmax_route_sparsemax_is_sparse_and_matches(ssa):
     assert cn[0, :, 5:].mean() < 8  # sparse: far fewer blocks than candidates
 
 
-@pytest.mark.parametrize("sigma,dtype,d,B", [(0.0, "bf16", 128, 64), (0.7, "bf16", 128, 64),
-                                             (1.0, "f32", 64, 32), (0.5, "bf16", 64, 16)])
-def test_prior_attention_parity(ssa, sigma, dtype, d, B):
+@pytest.mark.parametrize("sigma,dtype,d,B,Hq", [
+    (0.0, "bf16", 128, 64, 4), (0.7, "bf16", 128, 64, 4), (1.0, "f32", 64, 32, 4),
+    (0.5, "bf16", 64, 16, 4),
+    # the tensor-core kernel (bf16, d = 128, (Hq / Hkv) * B a multiple of 256)
+    (0.7, "bf16", 128, 64, 8), (1.0, "bf16", 128, 128, 4), (0.0, "bf16", 128, 64, 8)])
+def test_prior_attention_parity(ssa, sigma, dtype, d, B, Hq):
     N = B * 12 + 17
-    Q, K, V = planted_prefill(1, 4, 2, N, d, B, 3, seed=53, dtype=dtype)
+    Q, K, V = planted_prefill(1, Hq, 2, N, d, B, 3, seed=53, dtype=dtype)
     Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
     S = ssa.ssa_block_summary(Kd, B)
     idx, cnt, bias, w = ssa.ssa_route_entmax(Qd, S, B, 2, 1.5, 8.0, sigma, want_w=True)
@@ -116,17 +119,18 @@ def test_prior_attention_parity(ssa, sigma, dtype, d, B):
     np.testing.assert_allclose(to_f64(lse), rlse, rtol=0, atol=1e-4)
 
 
-def test_prior_attention_with_zero_sigma_is_topk_attention_on_the_support(ssa):
+@pytest.mark.parametrize("Hq,d", [(4, 64), (8, 128)])  # (8, 128): the tensor-core kernel
+def test_prior_attention_with_zero_sigma_is_topk_attention_on_the_support(ssa, Hq, d):
     # sigma = 0: no prior, so the result is the plain selected-block attention
-    # over the entmax support plus the diagonal -- bitwise the SIMT kernel of
+    # over the entmax support plus the diagonal -- bitwise the kernel of
     # ssa_sparse_attn_fwd run on the same block lists
-    B, N, d = 64, 64 * 10 + 3, 64
-    Q, K, V = planted_prefill(1, 4, 2, N, d, B, 3, seed=56, dtype="bf16")
+    B, N = 64, 64 * 10 + 3
+    Q, K, V = planted_prefill(1, Hq, 2, N, d, B, 3, seed=56, dtype="bf16")
     Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
     S = ssa.ssa_block_summary(Kd, B)
     idx, cnt, bias, _ = ssa.ssa_route_entmax(Qd, S, B, 2, 1.5, 8.0, 0.0)
     assert torch.all(bias == 0)
     a, la = ssa.ssa_sparse_attn_fwd_prior(Qd, Kd, Vd, idx, cnt, bias, B)
     b, lb = ssa.ssa_sparse_attn_fwd(Qd, Kd, Vd, idx, cnt, B)
-    assert not ssa.ssa_sparse_attn_uses_tensor_cores(torch.bfloat16, 4, 2, d, B)
+    assert ssa.ssa_sparse_attn_uses_tensor_cores(torch.bfloat16, Hq, 2, d, B) == (Hq == 8)
     assert torch.equal(a, b) and torch.equal(la, lb)
