@@ -14,7 +14,9 @@
 // TMEM (512 columns): tile t: S at 128 t, dP at 128 t + 64, dQ at 256 + 128 t.
 // Roles (320 threads): warp 0 TMA producer (Q and dO of the item, then K and V
 // of each chunk into a 2-stage ring); warp 1 TMEM owner and MMA issuer (one
-// thread); warps 2-5 tile 0, 6-9 tile 1, one thread per row (TMEM lane).
+// thread), which alternates the tiles so that one tile's dS is formed while
+// the other tile's MMAs run; warps 2-5 tile 0, 6-9 tile 1, one thread per row
+// (TMEM lane).
 // One work item per CTA.  Every mbarrier wait is bounded; on expiry the CTA
 // records SSA_ERR_TIMEOUT, stops issuing, drains what it issued and frees TMEM.
 #include <cuda.h>
@@ -200,31 +202,52 @@ __global__ void __launch_bounds__(kThreadsTc, 1) bwd_dq_tc_kernel(
       const uint32_t qa = ptx::smem_u32(Qs), ga = ptx::smem_u32(Gs);
       const uint32_t ka = ptx::smem_u32(Ks), va = ptx::smem_u32(Vs);
       bool ok = nch == 0 || wait_tc(&sh->q_full, 0, abort);
+      // S and dP of tile t for chunk c into TMEM (commits s_full[t])
+      auto issue_sdp = [&](int t, int c) {
+        const int s = c & 1;
+        ptx::tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t ok2 = (kk >> 2) * 8192 + (kk & 3) * 32;
+          ptx::mma_ss(tmem + t * 128, sdesc_tc(qa + t * kTileBytes + oq, 16, 1024),
+                      sdesc_tc(ka + s * kChunkBytes + ok2, 16, 1024), kIdescN64, kk > 0);
+          ptx::mma_ss(tmem + t * 128 + 64, sdesc_tc(ga + t * kTileBytes + oq, 16, 1024),
+                      sdesc_tc(va + s * kChunkBytes + ok2, 16, 1024), kIdescN64, kk > 0);
+        }
+        ptx::mma_commit(&sh->s_full[t]);
+      };
+      // dQ_t += dS_t K of chunk c (A = dS from TMEM, B = K MN-major)
+      auto issue_dq = [&](int t, int c) {
+        const int s = c & 1;
+        ptx::tc_fence_after();
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                      sdesc_tc(ka + s * kChunkBytes + kk * 2048, 8192, 1024), kIdescDQ,
+                      (c > 0 || kk > 0) ? 1u : 0u);
+      };
+      // The two tiles alternate: while one tile's dS is formed, the tensor
+      // cores run the other tile's dQ and next S / dP.  S / dP of chunk c + 1
+      // overwrite dS of chunk c, so they are issued after that dQ (MMAs of
+      // one thread run in issue order).
+      if (ok && nch > 0) {
+        if ((ok = wait_tc(&sh->kv_full[0], 0, abort))) {
+          issue_sdp(0, 0);
+          issue_sdp(1, 0);
+        }
+      }
       for (int c = 0; ok && c < nch; ++c) {
         const int s = c & 1;
-        if (!(ok = wait_tc(&sh->kv_full[s], (c >> 1) & 1, abort))) break;
-        ptx::tc_fence_after();
-        for (int t = 0; t < 2; ++t) {
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t ok2 = (kk >> 2) * 8192 + (kk & 3) * 32;
-            ptx::mma_ss(tmem + t * 128, sdesc_tc(qa + t * kTileBytes + oq, 16, 1024),
-                        sdesc_tc(ka + s * kChunkBytes + ok2, 16, 1024), kIdescN64, kk > 0);
-            ptx::mma_ss(tmem + t * 128 + 64, sdesc_tc(ga + t * kTileBytes + oq, 16, 1024),
-                        sdesc_tc(va + s * kChunkBytes + ok2, 16, 1024), kIdescN64, kk > 0);
-          }
-          ptx::mma_commit(&sh->s_full[t]);
+        const bool more = c + 1 < nch;
+        if (!(ok = wait_tc(&sh->p_full[0], c & 1, abort))) break;
+        issue_dq(0, c);
+        if (more) {
+          if (!(ok = wait_tc(&sh->kv_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort))) break;
+          issue_sdp(0, c + 1);
         }
-        for (int t = 0; t < 2; ++t) {
-          if (!(ok = wait_tc(&sh->p_full[t], c & 1, abort))) break;
-          ptx::tc_fence_after();
-          for (int kk = 0; kk < 4; ++kk)
-            ptx::mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                        sdesc_tc(ka + s * kChunkBytes + kk * 2048, 8192, 1024), kIdescDQ,
-                        (c > 0 || kk > 0) ? 1u : 0u);
-        }
-        if (!ok) break;
-        ptx::mma_commit(&sh->kv_empty[s]);
+        if (!(ok = wait_tc(&sh->p_full[1], c & 1, abort))) break;
+        issue_dq(1, c);
+        ptx::mma_commit(&sh->kv_empty[s]);  // K(c), V(c) read by every MMA of chunk c
+        if (more) issue_sdp(1, c + 1);
       }
       if (ok && nch > 0) ptx::mma_commit(&sh->o_done);
       // every issued MMA completes before TMEM is freed
