@@ -567,6 +567,25 @@ __global__ void __launch_bounds__(256) bwd_sink_reduce_kernel(
   }
 }
 
+// The selection transposed: for every (bg, i) and entry j <= i of its row,
+// bit i of key block j's mask.  OR is order-free, so the masks do not depend
+// on scheduling.  mask is zeroed beforehand.
+__global__ void __launch_bounds__(256) bwd_hitmask_kernel(const int32_t* __restrict__ idx,
+                                                          const int32_t* __restrict__ cnt,
+                                                          int nbg, int nq, int max_sel, int nwin,
+                                                          uint32_t* __restrict__ mask) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (long long)nbg * nq) return;
+  const int bg = (int)(t / nq), i = (int)(t - (long long)bg * nq);
+  const int ns = min(max(cnt[t], 0), max_sel);
+  const int32_t* row = idx + t * max_sel;
+  for (int e = 0; e < ns; ++e) {
+    const int j = row[e];
+    if (j >= 0 && j <= i)
+      atomicOr(&mask[((long long)bg * nq + j) * nwin + (i >> 5)], 1u << (i & 31));
+  }
+}
+
 size_t attn_bwd_smem_bytes(int d, int B) {
   return (size_t)6 * B * d * 2 + (size_t)4 * B * sizeof(float);
 }
@@ -580,8 +599,10 @@ BwdPlan plan_bwd(int batch, int Hq, int Hkv, int N, int d, int B) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   p.off_delta = 0;
   p.off_part = up((size_t)batch * Hq * N * sizeof(float));
-  p.bytes = up(p.off_part +
-               (size_t)batch * Hkv * p.sink_nsplit * 2 * (size_t)B * d * sizeof(float));
+  p.off_mask = up(p.off_part +
+                  (size_t)batch * Hkv * p.sink_nsplit * 2 * (size_t)B * d * sizeof(float));
+  p.nwin = (attn_tc_supported(SSA_BF16, Hq, Hkv, d, B) && B == 64) ? (nq + 31) / 32 : 0;
+  p.bytes = up(p.off_mask + (size_t)batch * Hkv * nq * p.nwin * sizeof(uint32_t));
   return p;
 }
 
@@ -617,9 +638,18 @@ static cudaError_t launch_bwd_t(const BwdPlan& pl, const void* Q, const void* K,
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return e;
-  if (tc && B == 64) {
-    e = launch_bwd_dkv_tc(Q, K, V, dO, lse, delta, idx, cnt, batch, Hq, Hkv, N, max_sel, scale,
-                          dK, dV, part, pl.sink_qr, pl.sink_nsplit, st);
+  if (tc && B == 64 && pl.nwin > 0) {
+    uint32_t* mask = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + pl.off_mask);
+    const size_t mbytes = (size_t)nbg * nq * pl.nwin * sizeof(uint32_t);
+    e = cudaMemsetAsync(mask, 0, mbytes, st);
+    if (e != cudaSuccess) return e;
+    const long long rows_bg = (long long)nbg * nq;
+    bwd_hitmask_kernel<<<(unsigned)((rows_bg + 255) / 256), 256, 0, st>>>(idx, cnt, nbg, nq,
+                                                                          max_sel, pl.nwin, mask);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = launch_bwd_dkv_tc(Q, K, V, dO, lse, delta, batch, Hq, Hkv, N, scale, dK, dV, part,
+                          pl.sink_qr, pl.sink_nsplit, mask, pl.nwin, st);
   } else {
     e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);

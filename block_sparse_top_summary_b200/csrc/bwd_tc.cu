@@ -270,7 +270,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) bwd_dq_tc_kernel(
     const bool valid = pos < N;
     const float l2 = valid ? lse[rowi] * kLog2eTc : INFINITY;
     const float dl = valid ? delta[rowi] : 0.f;
-    const float c2 = scale * kLog2eTc;
+    const uint64_t c2 = ptx::f2_pack(scale * kLog2eTc, scale * kLog2eTc);
+    const uint64_t nl2 = ptx::f2_pack(-l2, -l2), ndl = ptx::f2_pack(-dl, -dl);
     bool ok = true;
     for (int c = 0; c < nch; ++c) {
       if (!(ok = warp_wait_tc(&sh->s_full[t], c & 1, abort))) break;
@@ -283,18 +284,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1) bwd_dq_tc_kernel(
         ptx::tmem_ld32(tS + q * 32, sv);
         ptx::tmem_ld32(tS + 64 + q * 32, pv);
         ptx::tmem_wait_ld();
+        const int kmax = pos - k0 - q * 32;  // columns past it are keys after the query
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float ds[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int k = q * 32 + 2 * e + u;
-            const float p = (k0 + k <= pos)
-                                ? exp2f(fmaf(__uint_as_float(sv[2 * e + u]), c2, -l2))
-                                : 0.f;
-            ds[u] = p * (__uint_as_float(pv[2 * e + u]) - dl);
-          }
-          wv[q * 16 + e] = pack_bf16_tc(ds[0], ds[1]);
+          float p0, p1, d0, d1;
+          ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(sv[2 * e]),
+                                                  __uint_as_float(sv[2 * e + 1])),
+                                     c2, nl2),
+                         p0, p1);
+          p0 = 2 * e <= kmax ? ptx::ex2_ftz(p0) : 0.f;
+          p1 = 2 * e + 1 <= kmax ? ptx::ex2_ftz(p1) : 0.f;
+          ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(p0, p1),
+                                     ptx::f2_add(ptx::f2_pack(__uint_as_float(pv[2 * e]),
+                                                              __uint_as_float(pv[2 * e + 1])),
+                                                 ndl)),
+                         d0, d1);
+          wv[q * 16 + e] = pack_bf16_tc(d0, d1);
         }
       }
       // dS words over the first 32 S columns of this row (already read)
@@ -394,11 +399,20 @@ int read_and_reset_bwd_tc_error() {
 
 
 // ---------------------------------------------------------------- dK, dV
-
+// One CTA per (batch, KV head, key block j) at B = 64, over every query block
+// i whose selection holds j, 128 query rows (two heads) per step:
+//   S = Q K^T, dP = dO V^T      (M = 128 rows, N = 64 keys) into TMEM, 2 buffers
+//   P, dS as bf16 rows (128-byte swizzle) into shared memory, 2 buffers
+//   dV^T += dO^T P, dK^T += Q^T dS   (M = d = 128, N = 64; A and B MN-major)
+// Roles (320 threads): warp 0 TMA producer (K and V once, Q and dO per step
+// into a 2-stage ring); warp 1 TMEM owner and MMA issuer, S and dP one step
+// ahead of dV and dK; warps 2-9 form P and dS, two warps per TMEM lane
+// quarter, one per half of the keys, so a step's P and dS are formed while
+// the previous step's dV / dK MMAs run.
 
 namespace {
 
-constexpr int kThreadsKv = 192;
+constexpr int kThreadsKv = 320;
 constexpr uint32_t kTile = 32768;    // 128 rows x 128 d x 2 B (Q or dO)
 constexpr uint32_t kBlk = 16384;     // 64 keys x 128 d x 2 B (K or V)
 constexpr uint32_t kPd = 16384;      // 128 query rows x 64 keys x 2 B (P or dS)
@@ -409,8 +423,8 @@ struct __align__(8) SharedKv {
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2];
   uint64_t s_full[2];
-  uint64_t pd_full;   // P and dS of the step are in shared memory (128 arrivals)
-  uint64_t pd_empty;  // the step's dV / dK MMAs are done reading them
+  uint64_t pd_full[2];   // P and dS of the step are in shared memory (256 arrivals)
+  uint64_t pd_empty[2];  // the step's dV / dK MMAs are done reading them
   uint64_t done, drain;
   uint32_t tmem_base;
   int abort;
@@ -462,39 +476,15 @@ __device__ __forceinline__ uint32_t pk(float lo, float hi) {
   return r;
 }
 
-// Warp scan of the query blocks in [base, min(base + 32, end)): the mask of
-// those whose ascending selection row holds key block j.
-__device__ __forceinline__ unsigned hits32(const int32_t* idx_bg, const int32_t* cnt_bg, int end,
-                                           int max_sel, int j, int base) {
-  const int qi = base + (threadIdx.x & 31);
-  bool hit = false;
-  if (qi < end) {
-    const int32_t* row = idx_bg + (int64_t)qi * max_sel;
-    int lo = 0, hi = min(max(cnt_bg[qi], 0), max_sel);
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      const int v = row[mid];
-      if (v == j) {
-        hit = true;
-        break;
-      }
-      if (v < j) lo = mid + 1;
-      else hi = mid;
-    }
-  }
-  return __ballot_sync(0xffffffffu, hit);
-}
-
 }  // namespace
 
 __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-    const float* __restrict__ lse, const float* __restrict__ delta,
-    const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int batch, int Hq,
-    int Hkv, int N, int nq, int max_sel, float scale, __nv_bfloat16* __restrict__ dK,
-    __nv_bfloat16* __restrict__ dV, float* __restrict__ sink_part, int sink_qr,
-    int sink_nsplit) {
+    const float* __restrict__ lse, const float* __restrict__ delta, int batch, int Hq, int Hkv,
+    int N, int nq, float scale, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
+    float* __restrict__ sink_part, int sink_qr, int sink_nsplit,
+    const uint32_t* __restrict__ hitmask, int nwin) {
   constexpr int B = 64;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
@@ -503,27 +493,29 @@ __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
   unsigned char* Vs = Ks + kBlk;
   unsigned char* Qs = Vs + kBlk;          // 2 stages
   unsigned char* Gs = Qs + 2 * kTile;     // 2 stages
-  unsigned char* Ps = Gs + 2 * kTile;     // P
-  unsigned char* Ds = Ps + kPd;           // dS
-  SharedKv* sh = reinterpret_cast<SharedKv*>(Ds + kPd);
+  unsigned char* Ps = Gs + 2 * kTile;     // P, 2 buffers
+  unsigned char* Ds = Ps + 2 * kPd;       // dS, 2 buffers
+  SharedKv* sh = reinterpret_cast<SharedKv*>(Ds + 2 * kPd);
 
   const int nbg = batch * Hkv;
-  // CTAs [0, nbg * sink_nsplit) take the sink column (key block 0, in every
-  // selection) in ranges of sink_qr query blocks and write fp32 partial sums;
-  // the others take one key block j >= 1 each over every query block i >= j.
-  const int nsink = nbg * sink_nsplit;
-  const bool sink = (int)blockIdx.x < nsink;
-  int j, bg, i_lo, i_hi;
+  // The CTAs of one (batch, KV head) pair are consecutive, so the Q and dO
+  // tiles that the running CTAs re-read are one pair's (L2-sized) rather than
+  // every pair's.  Within a pair: sink_nsplit CTAs take the sink column (key
+  // block 0, in every selection) in ranges of sink_qr query blocks and write
+  // fp32 partial sums; then one CTA per key block j >= 1 over every query
+  // block i >= j, early (most selected) blocks first.
+  const int per_bg = sink_nsplit + nq - 1;
+  const int bg = blockIdx.x / per_bg;
+  const int r_bg = blockIdx.x - bg * per_bg;
+  const bool sink = r_bg < sink_nsplit;
+  const int rg = r_bg;  // sink range (sink CTAs only)
+  int j, i_lo, i_hi;
   if (sink) {
-    const int rg = blockIdx.x / nbg;
     j = 0;
-    bg = blockIdx.x - rg * nbg;
     i_lo = rg * sink_qr;
     i_hi = min(nq, i_lo + sink_qr);
   } else {
-    const int u = blockIdx.x - nsink;
-    j = 1 + u / nbg;
-    bg = u - (j - 1) * nbg;
+    j = 1 + (r_bg - sink_nsplit);
     i_lo = j;
     i_hi = nq;
   }
@@ -532,8 +524,14 @@ __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
   const int tiles = G / 2;  // 128-row tiles per query block: two heads each
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &sh->abort;
-  const int32_t* idx_bg = idx + (int64_t)bg * nq * max_sel;
-  const int32_t* cnt_bg = cnt + (int64_t)bg * nq;
+  const uint32_t* mrow = hitmask + ((int64_t)bg * nq + j) * nwin;
+  auto win_bits = [&](int base) -> unsigned {
+    unsigned m = __ldg(mrow + (base >> 5));
+    const int lo = i_lo - base, hi = i_hi - base;
+    if (lo > 0) m &= lo >= 32 ? 0u : (~0u << lo);
+    if (hi < 32) m &= hi <= 0 ? 0u : ((1u << hi) - 1u);
+    return m;
+  };
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&sh->kv_full, 1);
@@ -542,8 +540,10 @@ __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
       ptx::mbar_init(&sh->qd_empty[s], 1);
       ptx::mbar_init(&sh->s_full[s], 1);
     }
-    ptx::mbar_init(&sh->pd_full, 128);
-    ptx::mbar_init(&sh->pd_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&sh->pd_full[s], 256);
+      ptx::mbar_init(&sh->pd_empty[s], 1);
+    }
     ptx::mbar_init(&sh->done, 1);
     ptx::mbar_init(&sh->drain, 1);
     sh->abort = 0;
@@ -569,8 +569,8 @@ __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
     }
     int n = 0;
     bool ok = true;
-    for (int base_i = i_lo; ok && base_i < i_hi; base_i += 32) {
-      unsigned m = hits32(idx_bg, cnt_bg, i_hi, max_sel, j, base_i);
+    for (int base_i = i_lo & ~31; ok && base_i < i_hi; base_i += 32) {
+      unsigned m = win_bits(base_i);
       while (ok && m) {
         const int i = base_i + __ffs(m) - 1;
         m &= m - 1;
@@ -626,34 +626,66 @@ __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
           ptx::mma_ss(tmem + 256, sd(ga + s * kTile + kk * 2048, 16384, 1024),
-                      sd(pa + kk * 2048, 16384, 1024), kIdT, acc);
+                      sd(pa + s * kPd + kk * 2048, 16384, 1024), kIdT, acc);
           ptx::mma_ss(tmem + 320, sd(qa + s * kTile + kk * 2048, 16384, 1024),
-                      sd(da + kk * 2048, 16384, 1024), kIdT, acc);
+                      sd(da + s * kPd + kk * 2048, 16384, 1024), kIdT, acc);
         }
-        ptx::mma_commit(&sh->pd_empty);
+        ptx::mma_commit(&sh->pd_empty[s]);
         ptx::mma_commit(&sh->qd_empty[s]);
       }
       __syncwarp();
     };
-    // S / dP run one step ahead of dV / dK
-    for (int base_i = i_lo; ok && base_i < i_hi; base_i += 32) {
-      unsigned m = hits32(idx_bg, cnt_bg, i_hi, max_sel, j, base_i);
-      const int cnt_m = __popc(m);
-      for (int e = 0; ok && e < cnt_m * tiles; ++e) {
-        if (!(ok = warp_wkv(&sh->qd_full[n & 1], (n >> 1) & 1, abort))) break;
-        issue_s(n);
-        ++n;
-        if (n >= 2) {
-          if (!(ok = warp_wkv(&sh->pd_full, m_done & 1, abort))) break;
-          issue_dkv(m_done);
-          ++m_done;
+    // S / dP of a step are issued once its Q and dO have landed and its TMEM
+    // buffer is free (the P / dS of step n - 2 formed); dV / dK of a step once
+    // its P and dS are in shared memory.  Neither waits for the other, so the
+    // Q / dO stage of step n is released (its dV / dK done) while the load of
+    // step n + 1 is still in flight.  Query blocks are found 32 at a time.
+    int known = 0;                // steps found so far
+    int next_i = i_lo & ~31;      // first query block not yet scanned
+    unsigned long long t_last = 0;
+    uint32_t idle = 0;
+    while (ok) {
+      if (n >= known && next_i < i_hi) {
+        known += __popc(win_bits(next_i)) * tiles;
+        next_i += 32;
+        continue;
+      }
+      if (m_done >= known) break;  // every window scanned, every step issued
+      bool progress = false;
+      if (n < known && n <= m_done + 1) {
+        int rdy = 0;
+        if (lane == 0) rdy = ptx::mbar_test_wait(&sh->qd_full[n & 1], (n >> 1) & 1) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, rdy, 0)) {
+          issue_s(n);
+          ++n;
+          progress = true;
         }
       }
-    }
-    if (ok && m_done < n) {
-      if ((ok = warp_wkv(&sh->pd_full, m_done & 1, abort))) {
-        issue_dkv(m_done);
-        ++m_done;
+      if (m_done < n) {
+        int rdy = 0;
+        if (lane == 0) rdy = ptx::mbar_test_wait(&sh->pd_full[m_done & 1], (m_done >> 1) & 1) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, rdy, 0)) {
+          issue_dkv(m_done);
+          ++m_done;
+          progress = true;
+        }
+      }
+      if (progress) {
+        idle = 0;
+      } else if ((++idle & 255u) == 1u) {
+        int stop = 0;
+        if (lane == 0) {
+          const unsigned long long now = gt();
+          if (idle == 1u) t_last = now;
+          if (*abort) {
+            stop = 1;
+          } else if (now - t_last > kWaitKv) {
+            *abort = 1;
+            atomicCAS(&g_bwd_tc_error, 0, (int)SSA_ERR_TIMEOUT);
+            stop = 1;
+          }
+        }
+        if (__shfl_sync(0xffffffffu, stop, 0)) ok = false;
       }
     }
     if (lane == 0) {
@@ -664,78 +696,126 @@ __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
     }
   } else {
     // ------------------------------------------------------------ query rows
+    // warps 2-9: two warps per TMEM lane quarter, each taking half of the
+    // step's 64 keys (q = key half)
     const int quarter = warp & 3;
+    const int q = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;  // query row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const float c2 = scale * kL2e;
-    unsigned char* prow = Ps + r * 128;
-    unsigned char* drow = Ds + r * 128;
-    int n = 0;
-    bool ok = true;
-    for (int base_i = i_lo; ok && base_i < i_hi; base_i += 32) {
-      unsigned m = hits32(idx_bg, cnt_bg, i_hi, max_sel, j, base_i);
-      while (ok && m) {
-        const int i = base_i + __ffs(m) - 1;
-        m &= m - 1;
-        for (int tt = 0; ok && tt < tiles; ++tt, ++n) {
-          const int s = n & 1;
-          const int h = g * G + tt * 2 + r / B;
-          const int pos = i * B + (r % B);
-          const int64_t rowi = ((int64_t)b * Hq + h) * N + pos;
-          const bool valid = pos < N;
-          const float l2 = valid ? lse[rowi] * kL2e : INFINITY;
-          const float dl = valid ? delta[rowi] : 0.f;
-          if (!(ok = warp_wkv(&sh->s_full[s], (n >> 1) & 1, abort))) break;
-          // the previous step's dV / dK MMAs are done with the P / dS tiles
-          if (n >= 1 && !(ok = warp_wkv(&sh->pd_empty, (n - 1) & 1, abort))) break;
-          ptx::tc_fence_after();
-#pragma unroll 1
-          for (int q = 0; q < 2; ++q) {
-            uint32_t sv[32], pv[32], pw[16], dw[16];
-            ptx::tmem_ld32(tmem + lane_off + s * 128 + q * 32, sv);
-            ptx::tmem_ld32(tmem + lane_off + s * 128 + 64 + q * 32, pv);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float p[2], d2[2];
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int k = q * 32 + 2 * e + u;
-                p[u] = (j * B + k <= pos) ? exp2f(fmaf(__uint_as_float(sv[2 * e + u]), c2, -l2))
-                                          : 0.f;
-                d2[u] = p[u] * (__uint_as_float(pv[2 * e + u]) - dl);
-              }
-              pw[e] = pk(p[0], p[1]);
-              dw[e] = pk(d2[0], d2[1]);
-            }
-            // keys 32 q .. 32 q + 31 are 16-byte chunks 4 q .. 4 q + 3 of the row
-#pragma unroll
-            for (int cl = 0; cl < 4; ++cl) {
-              const int sc = ((4 * q + cl) ^ (r & 7)) << 4;
-              *reinterpret_cast<uint4*>(prow + sc) =
-                  make_uint4(pw[4 * cl], pw[4 * cl + 1], pw[4 * cl + 2], pw[4 * cl + 3]);
-              *reinterpret_cast<uint4*>(drow + sc) =
-                  make_uint4(dw[4 * cl], dw[4 * cl + 1], dw[4 * cl + 2], dw[4 * cl + 3]);
-            }
-          }
-          ptx::fence_proxy_async_smem();  // generic writes before the MMAs read them
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(&sh->pd_full);
+    const uint64_t c2 = ptx::f2_pack(scale * kL2e, scale * kL2e);
+    // Steps in issue order: query blocks i ascending (set bits of the hit
+    // mask), then the two-head tiles t of each.  The next step's lse and
+    // delta are loaded one step ahead, so their latency overlaps this step.
+    int base = i_lo & ~31;
+    unsigned m = base < i_hi ? win_bits(base) : 0u;
+    int i = -1, t = tiles - 1;
+    auto advance = [&]() {
+      if (i >= 0 && t + 1 < tiles) {
+        ++t;
+        return;
+      }
+      t = 0;
+      while (m == 0u) {
+        base += 32;
+        if (base >= i_hi) {
+          i = -1;
+          return;
         }
+        m = win_bits(base);
+      }
+      i = base + __ffs(m) - 1;
+      m &= m - 1;
+    };
+    auto row_of = [&](int ii, int tt) -> int64_t {
+      return ((int64_t)b * Hq + g * G + tt * 2 + r / B) * N + ii * B + (r % B);
+    };
+    advance();
+    float lse_n = 0.f, dl_n = 0.f;
+    bool valid_n = false;
+    if (i >= 0) {
+      valid_n = i * B + (r % B) < N;
+      if (valid_n) {
+        lse_n = lse[row_of(i, t)];
+        dl_n = delta[row_of(i, t)];
       }
     }
-    // ---- epilogue: lane = d; dV[key][d] = dV^T[d][key], dK likewise (times scale)
-    if (ok && n > 0 && warp_wkv(&sh->done, 0, abort)) {
+    int n = 0;
+    bool ok = true;
+    while (ok && i >= 0) {
+      const int ci = i, s = n & 1;
+      const int pos = ci * B + (r % B);
+      const float l2 = valid_n ? lse_n * kL2e : INFINITY;
+      const float dl = valid_n ? dl_n : 0.f;
+      advance();
+      if (i >= 0) {
+        valid_n = i * B + (r % B) < N;
+        if (valid_n) {
+          lse_n = lse[row_of(i, t)];
+          dl_n = delta[row_of(i, t)];
+        }
+      }
+      if (!(ok = warp_wkv(&sh->s_full[s], (n >> 1) & 1, abort))) break;
+      // the dV / dK MMAs of step n - 2 are done with this P / dS buffer
+      if (n >= 2 && !(ok = warp_wkv(&sh->pd_empty[s], ((n >> 1) - 1) & 1, abort))) break;
       ptx::tc_fence_after();
+      unsigned char* prow = Ps + s * kPd + r * 128;
+      unsigned char* drow = Ds + s * kPd + r * 128;
+      uint32_t sv[32], pv[32], pw[16], dw[16];
+      ptx::tmem_ld32(tmem + lane_off + s * 128 + q * 32, sv);
+      ptx::tmem_ld32(tmem + lane_off + s * 128 + 64 + q * 32, pv);
+      ptx::tmem_wait_ld();
+      // only the diagonal block (i = j) has keys after the query
+      const int kmax = ci == j ? pos - j * B - q * 32 : 64;
+      const uint64_t nl2 = ptx::f2_pack(-l2, -l2), ndl = ptx::f2_pack(-dl, -dl);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        float p0, p1, d0, d1;
+        ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(sv[2 * e]),
+                                                __uint_as_float(sv[2 * e + 1])),
+                                   c2, nl2),
+                       p0, p1);
+        p0 = 2 * e <= kmax ? ptx::ex2_ftz(p0) : 0.f;
+        p1 = 2 * e + 1 <= kmax ? ptx::ex2_ftz(p1) : 0.f;
+        const uint64_t pp = ptx::f2_pack(p0, p1);
+        ptx::f2_unpack(ptx::f2_mul(pp, ptx::f2_add(ptx::f2_pack(__uint_as_float(pv[2 * e]),
+                                                                __uint_as_float(pv[2 * e + 1])),
+                                                   ndl)),
+                       d0, d1);
+        pw[e] = pk(p0, p1);
+        dw[e] = pk(d0, d1);
+      }
+      // keys 32 q .. 32 q + 31 are 16-byte chunks 4 q .. 4 q + 3 of the row
+#pragma unroll
+      for (int cl = 0; cl < 4; ++cl) {
+        const int sc = ((4 * q + cl) ^ (r & 7)) << 4;
+        *reinterpret_cast<uint4*>(prow + sc) =
+            make_uint4(pw[4 * cl], pw[4 * cl + 1], pw[4 * cl + 2], pw[4 * cl + 3]);
+        *reinterpret_cast<uint4*>(drow + sc) =
+            make_uint4(dw[4 * cl], dw[4 * cl + 1], dw[4 * cl + 2], dw[4 * cl + 3]);
+      }
+      ptx::fence_proxy_async_smem();  // generic writes before the MMAs read them
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&sh->pd_full[s]);
+      ++n;
+    }
+    // ---- epilogue: lane = d; dV[key][d] = dV^T[d][key], dK likewise (times scale)
+    // (a key block that no query block selects gets zeros)
+    const bool have = ok && n > 0 && warp_wkv(&sh->done, 0, abort);
+    if (have || (ok && n == 0)) {
       const int dd = r;
-#pragma unroll 1
-      for (int q = 0; q < 2; ++q) {
+      {
         uint32_t vv[32], kv[32];
-        ptx::tmem_ld32(tmem + lane_off + 256 + q * 32, vv);
-        ptx::tmem_ld32(tmem + lane_off + 320 + q * 32, kv);
-        ptx::tmem_wait_ld();
+        if (have) {
+          ptx::tc_fence_after();
+          ptx::tmem_ld32(tmem + lane_off + 256 + q * 32, vv);
+          ptx::tmem_ld32(tmem + lane_off + 320 + q * 32, kv);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) vv[e] = kv[e] = 0u;
+        }
         if (sink) {
-          float* pk = sink_part + ((size_t)(blockIdx.x / nbg) * nbg + bg) * 2 * B * 128;
+          float* pk = sink_part + ((size_t)rg * nbg + bg) * 2 * B * 128;
           float* pv = pk + (size_t)B * 128;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -766,10 +846,10 @@ __global__ void __launch_bounds__(kThreadsKv, 1) bwd_dkv_tc_kernel(
 }
 
 cudaError_t launch_bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO,
-                              const float* lse, const float* delta, const int32_t* idx,
-                              const int32_t* cnt, int batch, int Hq, int Hkv, int N,
-                              int max_sel, float scale, void* dK, void* dV, float* sink_part,
-                              int sink_qr, int sink_nsplit, cudaStream_t st) {
+                              const float* lse, const float* delta, int batch, int Hq, int Hkv,
+                              int N, float scale, void* dK, void* dV, float* sink_part,
+                              int sink_qr, int sink_nsplit, const uint32_t* hitmask, int nwin,
+                              cudaStream_t st) {
   CUtensorMap mq, mg, mk, mv;
   if (!make_bf16_map(&mq, Q, 128, N, batch * Hq, 64) ||
       !make_bf16_map(&mg, dO, 128, N, batch * Hq, 64) ||
@@ -779,13 +859,13 @@ cudaError_t launch_bwd_dkv_tc(const void* Q, const void* K, const void* V, const
   const int nq = (N + 63) / 64;
   const long long ctas = (long long)batch * Hkv * (sink_nsplit + nq - 1);
   if (ctas <= 0) return cudaSuccess;
-  const size_t smem = 1024 + 2 * (size_t)kBlk + 4 * (size_t)kTile + 2 * (size_t)kPd + sizeof(SharedKv);
+  const size_t smem = 1024 + 2 * (size_t)kBlk + 4 * (size_t)kTile + 4 * (size_t)kPd + sizeof(SharedKv);
   cudaError_t e = cudaFuncSetAttribute(bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   bwd_dkv_tc_kernel<<<(unsigned)ctas, kThreadsKv, smem, st>>>(
-      mq, mg, mk, mv, lse, delta, idx, cnt, batch, Hq, Hkv, N, nq, max_sel, scale,
-      (__nv_bfloat16*)dK, (__nv_bfloat16*)dV, sink_part, sink_qr, sink_nsplit);
+      mq, mg, mk, mv, lse, delta, batch, Hq, Hkv, N, nq, scale, (__nv_bfloat16*)dK,
+      (__nv_bfloat16*)dV, sink_part, sink_qr, sink_nsplit, hitmask, nwin);
   return cudaGetLastError();
 }
 

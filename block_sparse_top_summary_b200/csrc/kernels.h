@@ -43,13 +43,17 @@ cudaError_t launch_entmax_route(const void* Q, ssa_dtype dt, const float* S, int
                                 float sigma, int max_sel, int32_t* idx, int32_t* cnt,
                                 float* bias, float* w, cudaStream_t st);
 
-// Backward pass of stage 2 (bf16, mma.sync tiles): delta, dQ, dK, dV.  The
-// workspace holds delta ([batch, Hq, N] fp32) and the sink column's partial
-// sums ([sink_nsplit][batch * Hkv][2][B][d] fp32).
+// Backward pass of stage 2: delta, dQ, dK, dV.  The workspace holds delta
+// ([batch, Hq, N] fp32), the sink column's partial sums
+// ([sink_nsplit][batch * Hkv][2][B][d] fp32) and, for the tensor-core dK / dV
+// pass, the selection transposed as bit masks: word w of (bg, key block j)
+// has bit t set when query block 32 w + t selects j ([batch * Hkv][nq][nwin]
+// uint32, nwin = ceil(nq / 32); nwin = 0 when that pass is not used).
 struct BwdPlan {
   int sink_qr;      // query blocks per sink range
   int sink_nsplit;  // sink ranges per (batch, KV head)
-  size_t off_delta, off_part, bytes;
+  int nwin;         // mask words per key block (0: no mask)
+  size_t off_delta, off_part, off_mask, bytes;
 };
 BwdPlan plan_bwd(int batch, int Hq, int Hkv, int N, int d, int B);
 size_t attn_bwd_smem_bytes(int d, int B);
@@ -61,10 +65,10 @@ cudaError_t launch_bwd_dq_tc(const void* Q, const void* K, const void* V, const 
                              const int32_t* cnt, int batch, int Hq, int Hkv, int N, int B,
                              int max_sel, float scale, void* dQ, cudaStream_t st);
 cudaError_t launch_bwd_dkv_tc(const void* Q, const void* K, const void* V, const void* dO,
-                              const float* lse, const float* delta, const int32_t* idx,
-                              const int32_t* cnt, int batch, int Hq, int Hkv, int N,
-                              int max_sel, float scale, void* dK, void* dV, float* sink_part,
-                              int sink_qr, int sink_nsplit, cudaStream_t st);
+                              const float* lse, const float* delta, int batch, int Hq, int Hkv,
+                              int N, float scale, void* dK, void* dV, float* sink_part,
+                              int sink_qr, int sink_nsplit, const uint32_t* hitmask, int nwin,
+                              cudaStream_t st);
 cudaError_t launch_attn_bwd(const BwdPlan& pl, const void* Q, const void* K, const void* V,
                             const void* O, const void* dO, const float* lse, const int32_t* idx,
                             const int32_t* cnt, int batch, int Hq, int Hkv, int N, int d, int B,
