@@ -140,8 +140,8 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
 #pragma unroll
       for (int e = 0; e < SL; ++e) qs[q][e] = qbar[q * D + lane * SL + e];
     const float* Sg = S + (int64_t)bg * nfull * D + lane * SL;
-    for (int j0 = 1 + warp * 4; j0 <= ncand; j0 += 4 * (256 / 32)) {
-      float sv[4][SL];
+    // the summary rows of a warp step are loaded one step ahead
+    auto load_rows = [&](int j0, float (&sv)[4][SL]) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int j = min(j0 + c, ncand);
@@ -153,6 +153,13 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
           sv[c][0] = x.x; sv[c][1 % SL] = x.y;
         }
       }
+    };
+    constexpr int kStep = 4 * (256 / 32);
+    float sv[4][SL];
+    if (1 + warp * 4 <= ncand) load_rows(1 + warp * 4, sv);
+    for (int j0 = 1 + warp * 4; j0 <= ncand; j0 += kStep) {
+      float sn[4][SL];
+      if (j0 + kStep <= ncand) load_rows(j0 + kStep, sn);
       float v[32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -168,6 +175,10 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
       const int q = lane % TQ;
       const int j = j0 + c;
       if (j <= ncand) sc[q * sc_stride + (j - 1)] = dot * inv_sqrt_d;
+#pragma unroll
+      for (int c2 = 0; c2 < 4; ++c2)
+#pragma unroll
+        for (int e = 0; e < SL; ++e) sv[c2][e] = sn[c2][e];
     }
   }
   __syncthreads();
