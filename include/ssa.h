@@ -247,9 +247,12 @@ ssa_status ssa_route_hierarchical(const void* Q, ssa_dtype dtype, const float* S
  * entry ignored.  It holds delta and the partial sums of the sink block
  * (block 0, which every query block selects): its dK and dV are summed over
  * ranges of query blocks by separate CTAs, and the ranges are added in a
- * fixed order.  Calls that share a workspace must not overlap on the device.
- * The contractions run on mma.sync tensor-core tiles (bf16 in, fp32
- * accumulate); P and dS are rounded to bf16 as operands, outputs to bf16.
+ * fixed order; for d = 128, B = 64 and (Hq / Hkv) * B a multiple of 256 it
+ * also holds the selection transposed as per-key-block bit masks.  Calls that
+ * share a workspace must not overlap on the device.  The contractions run on
+ * tensor cores (tcgen05 with TMEM accumulators for the forward's tensor-core
+ * shapes, mma.sync tiles otherwise; bf16 in, fp32 accumulate); P and dS are
+ * rounded to bf16 as operands, outputs to bf16.
  */
 ssa_status ssa_sparse_attn_bwd(const void* Q, const void* K, const void* V, const void* O,
                                const void* dO, const float* lse, ssa_dtype dtype,
