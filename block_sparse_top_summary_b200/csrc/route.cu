@@ -15,7 +15,8 @@
 //      d/32 coordinates of each summary and of the 8 qbar rows, so one
 //      coalesced load feeds 8*d/32 FMAs; the 32 partial dot products of a
 //      warp step are reduced with a 31-shuffle butterfly that leaves dot
-//      product l in lane l; scores land in shared memory;
+//      product l in lane l; scores land in shared memory (phases 1 and 2 are
+//      route_tile::pool and route_tile::score);
 //   3. select: warp w selects for query block w of the tile with an exact
 //      4-pass radix select (ties to the lower index) and writes the ascending
 //      block list, and, when the caller asks for them, the block's row of
@@ -24,31 +25,11 @@
 // candidates).
 #include "common.cuh"
 #include "kernels.h"
+#include "route_tile.cuh"
 
 namespace ssa {
 
-namespace {
-
-constexpr int TQ = 8;  // query blocks per CTA (= warps per CTA)
-
-// Butterfly reduction of 32 per-lane values: afterwards lane l's v[0] holds
-// the warp-wide sum of value index l.
-__device__ __forceinline__ float reduce32_transpose(float (&v)[32]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int half = 16; half >= 1; half >>= 1) {
-    const bool upper = (lane & half) != 0;
-#pragma unroll
-    for (int k = 0; k < half; ++k) {
-      const float send = upper ? v[k] : v[k + half];
-      const float keep = upper ? v[k + half] : v[k];
-      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-    }
-  }
-  return v[0];
-}
-
-}  // namespace
+using route_tile::TQ;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
@@ -59,9 +40,6 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
                                                     int N, int B, int nq, int nfull, int topk,
                                                     int max_sel, int ntiles, int sc_stride,
                                                     float inv_sqrt_d) {
-  constexpr int EPC = Vec16<T>::n;
-  constexpr int CPR = D / EPC;
-  constexpr int SL = D / 32;  // summary coordinates per lane
   extern __shared__ __align__(16) float smem[];
   float* qbar = smem;                                        // [TQ][D]
   uint32_t* hist = reinterpret_cast<uint32_t*>(qbar + TQ * D);  // [TQ][256]
@@ -78,109 +56,12 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
   const int i0 = tile * TQ;
   const int i1 = min(i0 + TQ, nq);
 
-  // ---- 1. pool Q over (rows of the block) x (heads of the group): warp w
-  // pools query block i0 + w.  A warp load covers RPW whole rows (16-byte
-  // chunk cc of row rs); 16 loads are in flight per lane; rows meet by
-  // xor-shuffles at the end, so this phase needs no block barrier.
-  {
-    constexpr int LPR = CPR < 32 ? CPR : 32;  // lanes per row
-    constexpr int RPW = 32 / LPR;             // rows per warp load
-    constexpr int U = 16;                     // loads in flight per lane
-    const int qi = i0 + warp;
-    if (qi < i1) {
-      const int rows = min(B, N - qi * B);
-      const int R = G * rows;
-      const int cc = lane % LPR;
-      const int rs = lane / LPR;
-      float acc[EPC];
-#pragma unroll
-      for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
-      const T* blk = Q + ((int64_t)(b * Hq + g * G) * N + (int64_t)qi * B) * D + cc * EPC;
-      for (int r0 = rs; r0 < R; r0 += RPW * U) {
-        uint4 v[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int r = r0 + u * RPW;
-          if (r < R) {
-            const int h = r / rows;
-            v[u] = ldg16_stream(blk + ((int64_t)h * N + (r - h * rows)) * D);
-          } else {
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          float f[EPC];
-          unpack16(v[u], f, (const T*)nullptr);
-#pragma unroll
-          for (int e = 0; e < EPC; ++e) acc[e] += f[e];
-        }
-      }
-#pragma unroll
-      for (int o = LPR; o < 32; o <<= 1)
-#pragma unroll
-        for (int e = 0; e < EPC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
-      if (rs == 0) {
-        const float inv = 1.0f / (float)R;
-#pragma unroll
-        for (int e = 0; e < EPC; ++e) qbar[warp * D + cc * EPC + e] = acc[e] * inv;
-      }
-    }
-    // CPR > 32 (fp32, d = 128 has CPR = 32): one row per warp load covers d
-    static_assert(CPR <= 32, "a row must fit one warp load");
-    __syncthreads();
-  }
+  // ---- 1. pool Q over (rows of the block) x (heads of the group)
+  route_tile::pool<T, D>(Q, qbar, b, g, G, Hq, N, B, i0, i1);
 
   // ---- 2. scores for candidates j = 1 .. i1-2 against all TQ rows
   const int ncand = max(i1 - 2, 0);
-  {
-    float qs[TQ][SL];
-#pragma unroll
-    for (int q = 0; q < TQ; ++q)
-#pragma unroll
-      for (int e = 0; e < SL; ++e) qs[q][e] = qbar[q * D + lane * SL + e];
-    const float* Sg = S + (int64_t)bg * nfull * D + lane * SL;
-    // the summary rows of a warp step are loaded one step ahead
-    auto load_rows = [&](int j0, float (&sv)[4][SL]) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int j = min(j0 + c, ncand);
-        if (SL == 4) {
-          const float4 x = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)j * D));
-          sv[c][0] = x.x; sv[c][1] = x.y; sv[c][2 % SL] = x.z; sv[c][3 % SL] = x.w;
-        } else {
-          const float2 x = __ldg(reinterpret_cast<const float2*>(Sg + (int64_t)j * D));
-          sv[c][0] = x.x; sv[c][1 % SL] = x.y;
-        }
-      }
-    };
-    constexpr int kStep = 4 * (256 / 32);
-    float sv[4][SL];
-    if (1 + warp * 4 <= ncand) load_rows(1 + warp * 4, sv);
-    for (int j0 = 1 + warp * 4; j0 <= ncand; j0 += kStep) {
-      float sn[4][SL];
-      if (j0 + kStep <= ncand) load_rows(j0 + kStep, sn);
-      float v[32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int q = 0; q < TQ; ++q) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < SL; ++e) a = fmaf(sv[c][e], qs[q][e], a);
-          v[c * TQ + q] = a;
-        }
-      const float dot = reduce32_transpose(v);
-      const int c = lane / TQ;
-      const int q = lane % TQ;
-      const int j = j0 + c;
-      if (j <= ncand) sc[q * sc_stride + (j - 1)] = dot * inv_sqrt_d;
-#pragma unroll
-      for (int c2 = 0; c2 < 4; ++c2)
-#pragma unroll
-        for (int e = 0; e < SL; ++e) sv[c2][e] = sn[c2][e];
-    }
-  }
+  route_tile::score<D>(qbar, S, sc, sc_stride, (int64_t)bg * nfull, 1, ncand, inv_sqrt_d);
   __syncthreads();
 
   // ---- 3. per query block: top-k, then {0} U R U {i} ascending, -1 padded

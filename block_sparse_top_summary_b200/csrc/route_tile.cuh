@@ -1,0 +1,152 @@
+// Phases shared by the routing kernels that take query blocks in tiles of
+// TQ = 8 (one warp each), 256 threads per CTA: pooling the tile's query
+// blocks, and scoring a range of block summaries against all of them.
+#pragma once
+
+#include "common.cuh"
+
+namespace ssa {
+namespace route_tile {
+
+constexpr int TQ = 8;         // query blocks per CTA (= warps per CTA)
+constexpr int kThreads = 256;
+
+// Butterfly reduction of 32 per-lane values: afterwards lane l's v[0] holds
+// the warp-wide sum of value index l.
+__device__ __forceinline__ float reduce32_transpose(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float send = upper ? v[k] : v[k + half];
+      const float keep = upper ? v[k + half] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
+// qbar[w] = mean of Q over the rows of query block i0 + w and the G heads of
+// KV head g, for the tile's query blocks [i0, i1).  Warp w pools query block
+// i0 + w: a warp load covers RPW whole rows (16-byte chunk cc of row rs), 16
+// loads are in flight per lane, and rows meet by xor-shuffles at the end, so
+// no block barrier is needed inside.  Ends with a block barrier.
+template <typename T, int D>
+__device__ __forceinline__ void pool(const T* __restrict__ Q, float* qbar, int b, int g, int G,
+                                     int Hq, int N, int B, int i0, int i1) {
+  constexpr int EPC = Vec16<T>::n;
+  constexpr int CPR = D / EPC;
+  constexpr int LPR = CPR < 32 ? CPR : 32;  // lanes per row
+  constexpr int RPW = 32 / LPR;             // rows per warp load
+  constexpr int U = 16;                     // loads in flight per lane
+  static_assert(CPR <= 32, "a row must fit one warp load");
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int qi = i0 + warp;
+  if (qi < i1) {
+    const int rows = min(B, N - qi * B);
+    const int R = G * rows;
+    const int cc = lane % LPR;
+    const int rs = lane / LPR;
+    float acc[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+    const T* blk = Q + ((int64_t)(b * Hq + g * G) * N + (int64_t)qi * B) * D + cc * EPC;
+    for (int r0 = rs; r0 < R; r0 += RPW * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int r = r0 + u * RPW;
+        if (r < R) {
+          const int h = r / rows;
+          v[u] = ldg16_stream(blk + ((int64_t)h * N + (r - h * rows)) * D);
+        } else {
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float f[EPC];
+        unpack16(v[u], f, (const T*)nullptr);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+      }
+    }
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (rs == 0) {
+      const float inv = 1.0f / (float)R;
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) qbar[warp * D + cc * EPC + e] = acc[e] * inv;
+    }
+  }
+  __syncthreads();
+}
+
+// sc[q * stride + (j - jlo)] = qbar[q] . S[bg, j] * inv_sqrt_d for j in
+// [jlo, jhi] and every row q of the tile.  Every warp takes 4 summaries at a
+// time; lane l holds d/32 coordinates of each summary and of the TQ qbar rows,
+// so one coalesced load feeds TQ*d/32 FMAs; the 32 partial dot products of a
+// warp step are reduced with a 31-shuffle butterfly that leaves dot product l
+// in lane l.  The summary rows of a step are loaded one step ahead.  No
+// barrier inside; the caller synchronises before reading sc.
+template <int D>
+__device__ __forceinline__ void score(const float* qbar, const float* __restrict__ S, float* sc,
+                                      int stride, int64_t srow0, int jlo, int jhi,
+                                      float inv_sqrt_d) {
+  constexpr int SL = D / 32;  // summary coordinates per lane
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  float qs[TQ][SL];
+#pragma unroll
+  for (int q = 0; q < TQ; ++q)
+#pragma unroll
+    for (int e = 0; e < SL; ++e) qs[q][e] = qbar[q * D + lane * SL + e];
+  const float* Sg = S + srow0 * D + lane * SL;
+  auto load_rows = [&](int j0, float (&sv)[4][SL]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = min(j0 + c, jhi);
+      if (SL == 4) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)j * D));
+        sv[c][0] = x.x; sv[c][1] = x.y; sv[c][2 % SL] = x.z; sv[c][3 % SL] = x.w;
+      } else {
+        const float2 x = __ldg(reinterpret_cast<const float2*>(Sg + (int64_t)j * D));
+        sv[c][0] = x.x; sv[c][1 % SL] = x.y;
+      }
+    }
+  };
+  constexpr int kStep = 4 * (kThreads / 32);
+  float sv[4][SL];
+  if (jlo + warp * 4 <= jhi) load_rows(jlo + warp * 4, sv);
+  for (int j0 = jlo + warp * 4; j0 <= jhi; j0 += kStep) {
+    float sn[4][SL];
+    if (j0 + kStep <= jhi) load_rows(j0 + kStep, sn);
+    float v[32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int q = 0; q < TQ; ++q) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < SL; ++e) a = fmaf(sv[c][e], qs[q][e], a);
+        v[c * TQ + q] = a;
+      }
+    const float dot = reduce32_transpose(v);
+    const int c = lane / TQ;
+    const int q = lane % TQ;
+    const int j = j0 + c;
+    if (j <= jhi) sc[q * stride + (j - jlo)] = dot * inv_sqrt_d;
+#pragma unroll
+    for (int c2 = 0; c2 < 4; ++c2)
+#pragma unroll
+      for (int e = 0; e < SL; ++e) sv[c2][e] = sn[c2][e];
+  }
+}
+
+}  // namespace route_tile
+}  // namespace ssa

@@ -214,7 +214,11 @@ ssa_status ssa_sparse_attn_fwd_prior(const void* Q, const void* K, const void* V
  *   - R = the top min(k_blk, pool size) of the pool by s_j (ties: lower
  *     index); selection = {0} U R U {i}, ascending, -1 padded.
  * M = 1 with k_seg >= nq is the flat ssa_route.  idx, cnt as for ssa_route,
- * with max_sel >= min(k_blk, nq) + 2.  k_seg <= 64.  One CTA per (b, g, i).
+ * with max_sel >= min(k_blk, nq) + 2.  k_seg <= 64.  Query blocks are taken
+ * in tiles of 8 per CTA with the pooling and scoring of ssa_route (the same
+ * fp32 scores, bitwise), while the tile's score rows fit in shared memory
+ * (about 6000 complete blocks with large M); beyond that one CTA per query
+ * block, whose sums run in another order.
  */
 ssa_status ssa_route_hierarchical(const void* Q, ssa_dtype dtype, const float* S, int batch,
                                   int Hq, int Hkv, int N, int d, int B, int M, int k_seg,
