@@ -419,13 +419,16 @@ def widened(ssa, p128, p32, q, Kc, Vc, Sc, L, cd, dev, stream, world, hbm_peak, 
     ms = time_call(f, 10, 3, stream, world)
     out["ssa_route_hierarchical"] = hbm(ms, p128.route_bytes(),
                                         describe(c) + ", segments of 8 blocks, 8 kept")
-    # DashAttention's stages on the 32K prefill
-    c = p32.c
+    # DashAttention's stages: the learned summary on the 128K keys (a stream,
+    # like the block summary), the routing and prior attention on the 32K prefill
+    c = p128.c
     qbar = torch.randn(c.Hkv, c.d, generator=gen, device=dev)
-    S_l = torch.empty_like(p32.S)
-    f = lambda: ssa.ssa_learned_summary(p32.K, qbar, c.B, S=S_l)
+    S_l = torch.empty_like(p128.S)
+    f = lambda: ssa.ssa_learned_summary(p128.K, qbar, c.B, S=S_l)
     ms = time_call(f, 20, 3, stream, world)
-    out["ssa_learned_summary"] = hbm(ms, p32.summary_bytes(), describe(c))
+    out["ssa_learned_summary"] = hbm(ms, p128.summary_bytes(), describe(c))
+    del S_l
+    c = p32.c
     f = lambda: ssa.ssa_route_entmax(p32.Q, p32.S, c.B, c.Hkv, 1.5, 8.0, 0.5)
     ms = time_call(f, 10, 3, stream, world)
     ei, ec, eb, _ = ssa.ssa_route_entmax(p32.Q, p32.S, c.B, c.Hkv, 1.5, 8.0, 0.5)

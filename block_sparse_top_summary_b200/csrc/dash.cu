@@ -19,12 +19,39 @@ namespace {
 __device__ __forceinline__ float to_float(float v) { return v; }
 __device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-constexpr int kSumRows = 8;       // key rows in flight per warp (learned summary)
+constexpr int kSumRows = 16;      // key rows in flight per warp (learned summary)
 constexpr int kRouteThreads = 256;
 constexpr int kBisect = 40;       // bisection steps on tau (interval 1 -> 2^-40)
 }  // namespace
 
-// One warp per (b, KV head, complete block); lane owns D / 32 columns.
+// E consecutive elements of one row, loaded as one vector of E * sizeof(T)
+// bytes (4, 8 or 16), widened to fp32 exactly.
+template <int E>
+__device__ __forceinline__ void load_row(const float* p, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    const float2 x = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = x.x; v[1] = x.y;
+  }
+}
+template <int E>
+__device__ __forceinline__ void load_row(const __nv_bfloat16* p, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(p));
+    bf16x2_to_f(x.x, v[0], v[1]);
+    bf16x2_to_f(x.y, v[2], v[3]);
+  } else {
+    const uint32_t x = __ldg(reinterpret_cast<const unsigned int*>(p));
+    bf16x2_to_f(x, v[0], v[1]);
+  }
+}
+
+// One warp per (b, KV head, complete block); lane owns D / 32 consecutive
+// columns.  kSumRows rows are loaded per step (one vector load each), their
+// logits are reduced together, and the step is folded into the online softmax
+// with one rescale to the step's new maximum.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) learned_summary_kernel(
     const T* __restrict__ K, const float* __restrict__ qbar, float* __restrict__ S, int Hkv,
@@ -47,10 +74,9 @@ __global__ void __launch_bounds__(256) learned_summary_kernel(
   for (int r0 = 0; r0 < B; r0 += kSumRows) {
     float k[kSumRows][E], z[kSumRows];
 #pragma unroll
-    for (int rr = 0; rr < kSumRows; ++rr) {
-      const int r = min(r0 + rr, B - 1);
+    for (int rr = 0; rr < kSumRows; ++rr) load_row<E>(base + (size_t)min(r0 + rr, B - 1) * D, k[rr]);
 #pragma unroll
-      for (int e = 0; e < E; ++e) k[rr][e] = to_float(base[(size_t)r * D + e]);
+    for (int rr = 0; rr < kSumRows; ++rr) {
       float a = 0.f;
 #pragma unroll
       for (int e = 0; e < E; ++e) a = fmaf(q[e], k[rr][e], a);
@@ -60,16 +86,23 @@ __global__ void __launch_bounds__(256) learned_summary_kernel(
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
       for (int rr = 0; rr < kSumRows; ++rr) z[rr] += __shfl_xor_sync(0xffffffffu, z[rr], o);
+    // one rescale per step: the step's rows against the running max
+    float mn = m;
+#pragma unroll
+    for (int rr = 0; rr < kSumRows; ++rr)
+      if (r0 + rr < B) mn = fmaxf(mn, z[rr]);
+    const float al = exp2f(m - mn);
+    l *= al;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] *= al;
 #pragma unroll
     for (int rr = 0; rr < kSumRows; ++rr) {
-      if (r0 + rr >= B) break;
-      const float mn = fmaxf(m, z[rr]);
-      const float al = exp2f(m - mn), p = exp2f(z[rr] - mn);
-      l = l * al + p;
+      const float p = r0 + rr < B ? exp2f(z[rr] - mn) : 0.f;
+      l += p;
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = fmaf(p, k[rr][e], acc[e] * al);
-      m = mn;
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(p, k[rr][e], acc[e]);
     }
+    m = mn;
   }
   float* out = S + (size_t)u * D + lane * E;
 #pragma unroll
