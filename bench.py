@@ -437,15 +437,15 @@ def widened(ssa, p128, p32, q, Kc, Vc, Sc, L, cd, dev, stream, world, hbm_peak, 
                                   mean_blocks=float(ec.float().mean()))
     Oe = torch.empty_like(p32.Q)
     f = lambda: ssa.ssa_sparse_attn_fwd_prior(p32.Q, p32.K, p32.V, ei, ec, eb, c.B, O=Oe)
-    ms = time_call(f, 3, 1, stream, world)
+    ms = time_call(f, 10, 3, stream, world)
     ecn = ec.cpu().numpy()
     fl = sum(attn_flops(ecn[b, g], c.N, c.B, c.Hq // c.Hkv, c.d)
              for b in range(c.batch) for g in range(c.Hkv))
     tf = fl / (ms * 1e-3) / 1e12
-    out["ssa_sparse_attn_fwd_prior"] = {"ms": ms, "TFLOP/s": tf, "bound": "alu",
+    out["ssa_sparse_attn_fwd_prior"] = {"ms": ms, "TFLOP/s": tf, "bound": "tensor",
                                         "flops": fl, "workload": describe(c) + ", entmax selection",
-                                        "note": "CUDA cores (FFMA); fraction of the bf16 tensor "
-                                                "peak given for scale only",
+                                        "note": "the tcgen05 attention kernel with the prior "
+                                                "as a per-block logit offset",
                                         **fracs(tf, bf16_peak, NOMINAL_BF16_TFLOPS)}
     return out
 
