@@ -332,7 +332,10 @@ ssa_status ssa_decode_per_head_workspace_size(int batch, int Hq, int Hkv, int Lm
   if (st != SSA_OK) return st;
   if (batch <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || topk < 0) return SSA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
-  *bytes = ssa::plan_decode(batch, Hq, Hq, d, B, topk, Lmax).bytes;
+  // the larger of the two layouts ssa_decode_per_head may use (it depends on the dtype)
+  const size_t a = ssa::plan_decode(batch, Hq, Hq, d, B, topk, Lmax).bytes;
+  const size_t u = ssa::plan_decode_union(batch, Hq, Hkv, d, B, topk, Lmax).bytes;
+  *bytes = a > u ? a : u;
   return SSA_OK;
 }
 
@@ -354,10 +357,21 @@ ssa_status ssa_decode_per_head(const void* q, const void* Kc, const void* Vc, ss
   if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(S) || !aligned16(O))
     return SSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSA_ERR_INVALID_ARG;
+  const size_t need_a = ssa::plan_decode(batch, Hq, Hq, d, B, topk, Lmax).bytes;
+  const size_t need_u = ssa::plan_decode_union(batch, Hq, Hkv, d, B, topk, Lmax).bytes;
+  if (ws_bytes < (need_a > need_u ? need_a : need_u)) return SSA_ERR_INVALID_ARG;
+  if (dtype == SSA_BF16 && Hq / Hkv <= 8) {
+    // One selection per query head; the split pass streams each KV head's
+    // union of its heads' blocks once, the heads that did not choose a block
+    // masked out of it.
+    const ssa::DecodePlan p = ssa::plan_decode_union(batch, Hq, Hkv, d, B, topk, Lmax);
+    return from_cuda(ssa::launch_decode(p, q, Kc, Vc, dtype, S, seqlens, batch, Hq, Hkv, Lmax, d,
+                                        B, scale, O, idx, workspace,
+                                        reinterpret_cast<cudaStream_t>(stream), ssa::CacheMap{}));
+  }
   // Every query head is its own unit: the grouped path with one query head
   // per unit, each unit reading the cache head h / (Hq / Hkv).
   const ssa::DecodePlan p = ssa::plan_decode(batch, Hq, Hq, d, B, topk, Lmax);
-  if (ws_bytes < p.bytes) return SSA_ERR_INVALID_ARG;
   ssa::CacheMap cm;
   cm.kv_div = Hq / Hkv;
   return from_cuda(ssa::launch_decode(p, q, Kc, Vc, dtype, S, seqlens, batch, Hq, Hq, Lmax, d, B,

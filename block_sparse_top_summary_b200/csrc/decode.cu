@@ -156,13 +156,58 @@ __device__ int block_select_topk(const float* sc, int n, int k, int first, int32
 
 }  // namespace
 
+// Scores of GG query heads against the summaries 1 .. n in one sweep: a warp
+// step takes 32 / GG summaries, lane l holding d/32 coordinates of each; the
+// butterfly leaves the dot product of (summary c, head h) in lane c GG + h.
+// Each dot product is formed in the order of the single-head sweep.
+// sc[h n + (j - 1)] for head h and summary j.
+template <int GG, int D>
+__device__ __forceinline__ void score_heads(const float* qg, const float* __restrict__ Sh, int n,
+                                            float* sc, float inv_sqrt_d) {
+  constexpr int SL = D / 32;
+  constexpr int CPS = 32 / GG;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float qs[GG][SL];
+#pragma unroll
+  for (int h = 0; h < GG; ++h)
+#pragma unroll
+    for (int e = 0; e < SL; ++e) qs[h][e] = qg[h * D + lane * SL + e];
+  const float* Sg = Sh + lane * SL;
+  for (int j0 = 1 + warp * CPS; j0 <= n; j0 += CPS * 8) {
+    float v[32];
+#pragma unroll
+    for (int c = 0; c < CPS; ++c) {
+      const int j = min(j0 + c, n);
+      float x[SL];
+      if constexpr (SL == 4) {
+        const float4 y = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)j * D));
+        x[0] = y.x; x[1] = y.y; x[2 % SL] = y.z; x[3 % SL] = y.w;
+      } else {
+        const float2 y = __ldg(reinterpret_cast<const float2*>(Sg + (int64_t)j * D));
+        x[0] = y.x; x[1 % SL] = y.y;
+      }
+#pragma unroll
+      for (int h = 0; h < GG; ++h) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < SL; ++e) a = fmaf(x[e], qs[h][e], a);
+        v[c * GG + h] = a;
+      }
+    }
+    const float dot = reduce32_transpose(v);
+    const int c = lane / GG, h = lane - (lane / GG) * GG;
+    const int j = j0 + c;
+    if (j <= n) sc[(size_t)h * n + (j - 1)] = dot * inv_sqrt_d;
+  }
+}
+
 // ---------------------------------------------------------------- 1. route
 template <typename T, int D>
 __global__ void __launch_bounds__(256, 2) decode_route_kernel(
     const T* __restrict__ q, const float* __restrict__ S, const int32_t* __restrict__ seqlens,
     int Hq, int Hkv, int Lmax, int B, int nsum, int kk, int width, int32_t* __restrict__ ws_idx,
     int32_t* __restrict__ ws_cnt, int* __restrict__ ws_ctr, int32_t* __restrict__ idx_out,
-    float inv_sqrt_d, int kv_div) {
+    float inv_sqrt_d, int kv_div, int head_width, int gsweep) {
   constexpr int SL = D / 32;
   extern __shared__ __align__(16) float smem[];
   float* qb = smem;                                          // [D]
@@ -179,13 +224,8 @@ __global__ void __launch_bounds__(256, 2) decode_route_kernel(
   const int n = valid ? max(last - 1, 0) : 0;  // candidates 1 .. last-1
   if (t == 0) ws_ctr[bg] = 0;                   // reset the split counter for pass 2
 
-  if (t < D) {
-    float s = 0.f;
-    for (int h = 0; h < G; ++h) s += (float)q[((int64_t)b * Hq + g * G + h) * D + t];
-    qb[t] = s / (float)G;
-  }
-  __syncthreads();
-  {
+  // scores of the candidates against qb, into sc
+  auto score = [&]() {
     float qs[SL];
 #pragma unroll
     for (int e = 0; e < SL; ++e) qs[e] = qb[lane * SL + e];
@@ -215,26 +255,90 @@ __global__ void __launch_bounds__(256, 2) decode_route_kernel(
       const int j = j0 + lane;
       if (j <= n) sc[j - 1] = dot * inv_sqrt_d;
     }
-  }
-  __syncthreads();
+  };
   __shared__ int sbuf[16];
   int32_t* row = ws_idx + (int64_t)bg * width;
-  int n_sel = 0;
-  if (valid) {
-    n_sel = 1;
-    if (last >= 1) {
-      const int m = block_select_topk(sc, n, kk, 1, row + 1, hist, sbuf);
-      if (t == 0) row[m + 1] = last;
-      n_sel = m + 2;
+  // {0} + top-k of the candidates (scores at scs) + {last} into row[0 ..);
+  // returns the count
+  auto select = [&](const float* scs) -> int {
+    int n_sel = 0;
+    if (valid) {
+      n_sel = 1;
+      if (last >= 1) {
+        const int m = block_select_topk(scs, n, kk, 1, row + 1, hist, sbuf);
+        if (t == 0) row[m + 1] = last;
+        n_sel = m + 2;
+      }
+      if (t == 0) row[0] = 0;
     }
-    if (t == 0) row[0] = 0;
+    return n_sel;
+  };
+
+  if (head_width == 0) {
+    // one selection per KV head from the group-mean query
+    if (t < D) {
+      float s = 0.f;
+      for (int h = 0; h < G; ++h) s += (float)q[((int64_t)b * Hq + g * G + h) * D + t];
+      qb[t] = s / (float)G;
+    }
+    __syncthreads();
+    score();
+    __syncthreads();
+    const int n_sel = select(sc);
+    for (int p = n_sel + t; p < width; p += 256) row[p] = -1;
+    if (t == 0) ws_cnt[bg] = n_sel;
+    __syncthreads();
+    if (idx_out != nullptr) {
+      for (int p = t; p < width; p += 256) idx_out[(int64_t)bg * width + p] = row[p];
+    }
+    return;
   }
-  for (int p = n_sel + t; p < width; p += 256) row[p] = -1;
-  if (t == 0) ws_cnt[bg] = n_sel;
+
+  // one selection per query head; the row then holds their union, ascending,
+  // each entry j | (mask of the heads that chose j) << 24
+  // (gsweep > 1: the G heads scored in one sweep over the summaries into
+  // sc[G][n]; else one sweep per head)
+  uint8_t* hm = reinterpret_cast<uint8_t*>(sc + (size_t)gsweep * (nsum > 0 ? nsum : 1));
+  float* qg = reinterpret_cast<float*>(hm + (((size_t)nsum + 2 + 15) & ~(size_t)15));  // [G][D]
+  for (int j = t; j < nsum + 2; j += 256) hm[j] = 0;
+  if (gsweep > 1) {
+    for (int e = t; e < G * D; e += 256) qg[e] = (float)q[((int64_t)b * Hq + g * G) * D + e];
+    __syncthreads();
+    const float* Sh = S + ((int64_t)b * Hkv + g) * nsum * D;
+    if (G == 2) score_heads<2, D>(qg, Sh, n, sc, inv_sqrt_d);
+    else if (G == 4) score_heads<4, D>(qg, Sh, n, sc, inv_sqrt_d);
+    else score_heads<8, D>(qg, Sh, n, sc, inv_sqrt_d);
+  }
+  for (int h = 0; h < G; ++h) {
+    __syncthreads();  // the previous head's list is consumed
+    if (gsweep == 1) {
+      if (t < D) qb[t] = (float)q[((int64_t)b * Hq + g * G + h) * D + t];
+      __syncthreads();
+      score();
+      __syncthreads();
+    }
+    const int n_sel = select(gsweep > 1 ? sc + (size_t)h * n : sc);
+    __syncthreads();
+    for (int p = t; p < n_sel; p += 256) hm[row[p]] |= (uint8_t)(1u << h);
+    if (idx_out != nullptr) {
+      int32_t* orow = idx_out + ((int64_t)b * Hq + g * G + h) * head_width;
+      for (int p = t; p < head_width; p += 256) orow[p] = p < n_sel ? row[p] : -1;
+    }
+  }
   __syncthreads();
-  if (idx_out != nullptr) {
-    for (int p = t; p < width; p += 256) idx_out[(int64_t)bg * width + p] = row[p];
+  __shared__ int wsum[8];
+  int total = 0;
+  const int nb = valid ? last + 1 : 0;  // blocks 0 .. last
+  for (int base = 0; base < nb; base += 256) {
+    const int j = base + t;
+    const int mask = j < nb ? (int)hm[j] : 0;
+    int tot = 0;
+    const int off = block_excl_scan(mask != 0 ? 1 : 0, wsum, &tot);
+    if (mask != 0) row[total + off] = j | (mask << 24);
+    total += tot;
   }
+  for (int p = total + t; p < width; p += 256) row[p] = -1;
+  if (t == 0) ws_cnt[bg] = total;
 }
 
 // -------------------------------------------------------- 2. split-KV attention
@@ -882,6 +986,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
     // tensor-map coordinates of a unit: row y, head z (contiguous: z = the
     // cache head b * Hc + gc; paged: y within the block's page, z = page * Hc
     // + gc)
+    // rows: the unit's key rows, with the mask of the query heads that chose
+    // the block in bits 16-23 (0: every head)
     auto resolve = [&](long long u, int& y, int& z, int& rows) {
       y = 0;
       z = 0;
@@ -891,7 +997,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
       const int rem = (int)(u - (long long)bg * Ubg);
       const int s = rem / subs, r = rem - s * subs;
       if (s >= ws_cnt[bg]) return;
-      const int j = ws_idx[(int64_t)bg * width + s];
+      const int ent = ws_idx[(int64_t)bg * width + s];
+      const int j = ent & 0xFFFFFF;
+      const int hmask = (int)((unsigned)ent >> 24);
       const int L = seqlens[bg / Hkv];
       const int k0 = j * B + r * CK;
       const int rr = min(CK, min(L, (j + 1) * B) - k0);
@@ -907,7 +1015,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
         y = k0;
         z = b * Hc + gc;
       }
-      rows = rr;
+      rows = rr | (hmask << 16);
     };
     int y_n, z_n, rows_n;
     resolve(u0 + lane, y_n, z_n, rows_n);
@@ -928,7 +1036,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
         if (lane == 0) {
           info[st] = rows;
           ptx::st_release_s32(&tag[st], n);
-          if (rows > 0) {
+          if ((rows & 0xFFFF) > 0) {
             unsigned char* dst = base + (size_t)st * stage_bytes;
             // whole boxes land (rows past the sequence are masked, rows past
             // the cache read as zeros), so the byte count is fixed
@@ -1067,7 +1175,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
     const int st = n % stages;
     if (warp_wait_tag(&tag[st], n, abort) &&
         warp_wait_bounded(&full[st], (uint32_t)(n / stages) & 1u, abort)) {
-      const int rows = info[st];
+      const int rows = info[st] & 0xFFFF;
+      const unsigned hmask = (unsigned)info[st] >> 16;
+      // a query head that did not choose this block sees none of its keys
+      const bool row_on = hmask == 0u || ((hmask >> gr) & 1u) != 0u;
       if (rows > 0) {
         unsigned char* stg = base + (size_t)st * stage_bytes;
         const uint32_t sK = ptx::smem_u32(stg);
@@ -1109,7 +1220,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int key = nt * 8 + 2 * tq + e;
-            const float x = key < rows ? sc[nt][e] * scale_log2 : -INFINITY;
+            const float x = (key < rows && row_on) ? sc[nt][e] * scale_log2 : -INFINITY;
             sc[nt][e] = x;
             cm = fmaxf(cm, x);
           }
@@ -1127,11 +1238,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_mma_kernel(
         }
         __syncwarp();  // reconverge before the warp-collective mma.sync below
         uint32_t pa[NT / 2][2];
+        // a row with no key yet (m_run = -inf) has every x = -inf here: P = 0
+        const float mr = m_run == -INFINITY ? 0.f : m_run;
 #pragma unroll
         for (int p = 0; p < NT / 2; ++p) {
-          const float p0 = ex2_approx(sc[2 * p][0] - m_run), p1 = ex2_approx(sc[2 * p][1] - m_run);
-          const float p2 = ex2_approx(sc[2 * p + 1][0] - m_run);
-          const float p3 = ex2_approx(sc[2 * p + 1][1] - m_run);
+          const float p0 = ex2_approx(sc[2 * p][0] - mr), p1 = ex2_approx(sc[2 * p][1] - mr);
+          const float p2 = ex2_approx(sc[2 * p + 1][0] - mr);
+          const float p3 = ex2_approx(sc[2 * p + 1][1] - mr);
           l_run += (p0 + p1) + (p2 + p3);
           pa[p][0] = pack_bf16x2(p0, p1);
           pa[p][1] = pack_bf16x2(p2, p3);
@@ -1201,6 +1314,27 @@ DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int L
   const StreamGeom s2 = stream_geom(bgn, p.width, d, B, 2);
   const StreamGeom s4 = stream_geom(bgn, p.width, d, B, 4);
   p.parts_max = s2.parts_max > s4.parts_max ? s2.parts_max : s4.parts_max;
+  const size_t bg = (size_t)bgn;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  p.off_idx = 0;
+  p.off_cnt = up(p.off_idx + bg * p.width * sizeof(int32_t));
+  p.off_ctr = up(p.off_cnt + bg * sizeof(int32_t));
+  p.off_part = up(p.off_ctr + bg * sizeof(int32_t));
+  p.bytes = up(p.off_part + bg * p.parts_max * (size_t)p.G * (d + 2) * sizeof(float));
+  return p;
+}
+
+DecodePlan plan_decode_union(int batch, int Hq, int Hkv, int d, int B, int topk, int Lmax) {
+  DecodePlan p{};
+  p.G = Hq / Hkv;
+  p.nblk_max = (Lmax + B - 1) / B;
+  p.kk = topk < p.nblk_max ? topk : p.nblk_max;
+  p.head_width = p.kk + 2;
+  const int uw = p.G * p.kk + 2;  // the union of the heads' lists (sink and last shared)
+  p.width = uw < p.nblk_max ? uw : (p.nblk_max > 2 ? p.nblk_max : 2);
+  const int bgn = batch * Hkv;
+  const StreamGeom s2 = stream_geom(bgn, p.width, d, B, 2);
+  p.parts_max = s2.parts_max;
   const size_t bg = (size_t)bgn;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   p.off_idx = 0;
@@ -1295,13 +1429,24 @@ static cudaError_t launch_decode_t(const DecodePlan& p, const void* q, const voi
   int* ws_ctr = reinterpret_cast<int*>(w + p.off_ctr);
   float* ws_part = reinterpret_cast<float*>(w + p.off_part);
   const int nsum = Lmax / B;
-  const size_t smem1 = sizeof(float) * (D + 256 + (size_t)(nsum > 0 ? nsum : 1));
+  // the union of the heads' selections is streamed by the bf16 split pass only,
+  // whose rows are the group's (at most 8) query heads
+  if (p.head_width > 0 && (sizeof(T) != 2 || p.G > 8 || pm.kv_div != 1)) return cudaErrorInvalidValue;
+  // union: the G heads' scores in one sweep when they fit beside the rest
+  const size_t nsc = (size_t)(nsum > 0 ? nsum : 1);
+  const int gsweep = (p.head_width > 0 && (p.G == 2 || p.G == 4 || p.G == 8) &&
+                      sizeof(float) * p.G * (nsc + D) <= (size_t)160 * 1024)
+                         ? p.G
+                         : 1;
+  const size_t smem1 = sizeof(float) * (D + 256 + gsweep * nsc) +
+                       (p.head_width > 0 ? (((size_t)nsum + 2 + 15) & ~(size_t)15) : 0) +
+                       (gsweep > 1 ? sizeof(float) * p.G * D : 0);
   cudaError_t e = cudaFuncSetAttribute(decode_route_kernel<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
   decode_route_kernel<T, D><<<batch * Hkv, 256, smem1, st>>>(
       (const T*)q, S, seqlens, Hq, Hkv, Lmax, B, nsum, p.kk, p.width, ws_idx, ws_cnt, ws_ctr,
-      idx_out, 1.0f / sqrtf((float)D), pm.kv_div);
+      idx_out, 1.0f / sqrtf((float)D), pm.kv_div, p.head_width, gsweep);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if constexpr (sizeof(T) == 2) {

@@ -96,10 +96,15 @@ struct DecodePlan {
   int kk;         // effective top-k: min(topk, nblk_max)
   int width;      // idx row width: kk + 2
   int parts_max;  // partial records per (sequence, KV head) the scratch holds
+  int head_width; // 0: one selection per KV head; else one per query head, of this width,
+                  // and the split pass streams their union (bf16, G <= 8)
   size_t off_idx, off_cnt, off_part, off_ctr, bytes;
 };
 
 DecodePlan plan_decode(int batch, int Hq, int Hkv, int d, int B, int topk, int Lmax);
+// One selection per query head; the KV head's scratch row holds the union of
+// its G heads' blocks, each entry j | (head mask << 24).
+DecodePlan plan_decode_union(int batch, int Hq, int Hkv, int d, int B, int topk, int Lmax);
 
 cudaError_t launch_decode(const DecodePlan& p, const void* q, const void* Kc, const void* Vc,
                           ssa_dtype dt, const float* S, const int32_t* seqlens, int batch, int Hq,
