@@ -320,7 +320,10 @@ ssa_status ssa_decode(const void* q, const void* Kc, const void* Vc, ssa_dtype d
  * and attends only its own selection, reading the cache head h / G.
  * idx: NULL or [batch, Hq, min(topk, ceil(Lmax / B)) + 2] int32 (written).
  * workspace: ssa_decode_per_head_workspace_size(...) bytes, 256-byte aligned.
- * Any G = Hq / Hkv (each unit holds one query row).
+ * Any G = Hq / Hkv.  For bf16 with G <= 8 the cache blocks of a KV head are
+ * streamed once for the union of its heads' selections, each head masked out
+ * of the blocks it did not choose; otherwise every query head is a unit of
+ * its own.
  */
 ssa_status ssa_decode_per_head_workspace_size(int batch, int Hq, int Hkv, int Lmax, int d, int B,
                                               int topk, size_t* bytes);
