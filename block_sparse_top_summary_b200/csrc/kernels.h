@@ -14,7 +14,7 @@ cudaError_t launch_block_summary(const void* K, ssa_dtype dt, int batch, int Hkv
 
 // Largest number of query blocks ssa_route handles (its score rows live in
 // shared memory).
-constexpr int kRouteMaxBlocks = 4096;
+constexpr int kRouteMaxBlocks = 16384;
 
 cudaError_t launch_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq, int Hkv,
                          int N, int d, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,

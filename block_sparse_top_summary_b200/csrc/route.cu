@@ -29,9 +29,7 @@
 
 namespace ssa {
 
-using route_tile::TQ;
-
-template <typename T, int D>
+template <typename T, int D, int TQ>
 __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
                                                     const float* __restrict__ S,
                                                     int32_t* __restrict__ idx,
@@ -61,7 +59,7 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
 
   // ---- 2. scores for candidates j = 1 .. i1-2 against all TQ rows
   const int ncand = max(i1 - 2, 0);
-  route_tile::score<D>(qbar, S, sc, sc_stride, (int64_t)bg * nfull, 1, ncand, inv_sqrt_d);
+  route_tile::score<D, TQ>(qbar, S, sc, sc_stride, (int64_t)bg * nfull, 1, ncand, inv_sqrt_d);
   __syncthreads();
 
   // ---- 3. per query block: top-k, then {0} U R U {i} ascending, -1 padded
@@ -92,24 +90,39 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
   }
 }
 
-template <typename T, int D>
-static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int Hq, int Hkv, int N,
-                                  int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
-                                  float* scores, cudaStream_t st) {
+template <typename T, int D, int TQ>
+static cudaError_t launch_route_tq(const void* Q, const float* S, int batch, int Hq, int Hkv,
+                                   int N, int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
+                                   float* scores, cudaStream_t st) {
   const int nq = (N + B - 1) / B;
   const int nfull = N / B;
   const int ntiles = (nq + TQ - 1) / TQ;
   const int sc_stride = nq > 2 ? nq - 2 : 1;
   const size_t smem = sizeof(float) * ((size_t)TQ * D + (size_t)TQ * 256 + (size_t)TQ * sc_stride);
-  cudaError_t e = cudaFuncSetAttribute(route_kernel<T, D>,
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<T, D, TQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(batch * Hkv, ntiles);
-  route_kernel<T, D><<<grid, 256, smem, st>>>((const T*)Q, S, idx, cnt, scores, Hq, Hkv, N, B,
-                                              nq, nfull,
-                                              topk, max_sel, ntiles, sc_stride,
-                                              1.0f / sqrtf((float)D));
+  route_kernel<T, D, TQ><<<grid, 256, smem, st>>>((const T*)Q, S, idx, cnt, scores, Hq, Hkv, N, B,
+                                                  nq, nfull, topk, max_sel, ntiles, sc_stride,
+                                                  1.0f / sqrtf((float)D));
   return cudaGetLastError();
+}
+
+// Tiles of 8 query blocks while their score rows fit in shared memory, else
+// 4 or 2 (the warps past the tile idle in the pooling and selection phases).
+template <typename T, int D>
+static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int Hq, int Hkv, int N,
+                                  int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
+                                  float* scores, cudaStream_t st) {
+  const int nq = (N + B - 1) / B;
+  const size_t row = sizeof(float) * ((size_t)D + 256 + (size_t)(nq > 2 ? nq - 2 : 1));
+  const size_t limit = (size_t)220 * 1024;
+  if (8 * row <= limit)
+    return launch_route_tq<T, D, 8>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt, scores, st);
+  if (4 * row <= limit)
+    return launch_route_tq<T, D, 4>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt, scores, st);
+  return launch_route_tq<T, D, 2>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt, scores, st);
 }
 
 cudaError_t launch_route(const void* Q, ssa_dtype dt, const float* S, int batch, int Hq, int Hkv,

@@ -1,6 +1,7 @@
 // Phases shared by the routing kernels that take query blocks in tiles of
-// TQ = 8 (one warp each), 256 threads per CTA: pooling the tile's query
-// blocks, and scoring a range of block summaries against all of them.
+// TQ (8, or 4 or 2 for long sequences; one warp each), 256 threads per CTA:
+// pooling the tile's query blocks, and scoring a range of block summaries
+// against all of them.
 #pragma once
 
 #include "common.cuh"
@@ -8,7 +9,7 @@
 namespace ssa {
 namespace route_tile {
 
-constexpr int TQ = 8;         // query blocks per CTA (= warps per CTA)
+constexpr int TQ = 8;         // query blocks per CTA (= warps per CTA) unless stated
 constexpr int kThreads = 256;
 
 // Butterfly reduction of 32 per-lane values: afterwards lane l's v[0] holds
@@ -88,28 +89,29 @@ __device__ __forceinline__ void pool(const T* __restrict__ Q, float* qbar, int b
 }
 
 // sc[q * stride + (j - jlo)] = qbar[q] . S[bg, j] * inv_sqrt_d for j in
-// [jlo, jhi] and every row q of the tile.  Every warp takes 4 summaries at a
-// time; lane l holds d/32 coordinates of each summary and of the TQ qbar rows,
-// so one coalesced load feeds TQ*d/32 FMAs; the 32 partial dot products of a
-// warp step are reduced with a 31-shuffle butterfly that leaves dot product l
-// in lane l.  The summary rows of a step are loaded one step ahead.  No
-// barrier inside; the caller synchronises before reading sc.
-template <int D>
+// [jlo, jhi] and every row q < NQ of the tile.  Every warp takes CW = 32 / NQ
+// summaries at a time; lane l holds d/32 coordinates of each summary and of
+// the NQ qbar rows, so one coalesced load feeds NQ*d/32 FMAs; the 32 partial
+// dot products of a warp step are reduced with a 31-shuffle butterfly that
+// leaves dot product l in lane l.  The summary rows of a step are loaded one
+// step ahead.  No barrier inside; the caller synchronises before reading sc.
+template <int D, int NQ = TQ>
 __device__ __forceinline__ void score(const float* qbar, const float* __restrict__ S, float* sc,
                                       int stride, int64_t srow0, int jlo, int jhi,
                                       float inv_sqrt_d) {
   constexpr int SL = D / 32;  // summary coordinates per lane
+  constexpr int CW = 32 / NQ; // summaries per warp step
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  float qs[TQ][SL];
+  float qs[NQ][SL];
 #pragma unroll
-  for (int q = 0; q < TQ; ++q)
+  for (int q = 0; q < NQ; ++q)
 #pragma unroll
     for (int e = 0; e < SL; ++e) qs[q][e] = qbar[q * D + lane * SL + e];
   const float* Sg = S + srow0 * D + lane * SL;
-  auto load_rows = [&](int j0, float (&sv)[4][SL]) {
+  auto load_rows = [&](int j0, float (&sv)[CW][SL]) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < CW; ++c) {
       const int j = min(j0 + c, jhi);
       if (SL == 4) {
         const float4 x = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)j * D));
@@ -120,29 +122,29 @@ __device__ __forceinline__ void score(const float* qbar, const float* __restrict
       }
     }
   };
-  constexpr int kStep = 4 * (kThreads / 32);
-  float sv[4][SL];
-  if (jlo + warp * 4 <= jhi) load_rows(jlo + warp * 4, sv);
-  for (int j0 = jlo + warp * 4; j0 <= jhi; j0 += kStep) {
-    float sn[4][SL];
+  constexpr int kStep = CW * (kThreads / 32);
+  float sv[CW][SL];
+  if (jlo + warp * CW <= jhi) load_rows(jlo + warp * CW, sv);
+  for (int j0 = jlo + warp * CW; j0 <= jhi; j0 += kStep) {
+    float sn[CW][SL];
     if (j0 + kStep <= jhi) load_rows(j0 + kStep, sn);
     float v[32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < CW; ++c)
 #pragma unroll
-      for (int q = 0; q < TQ; ++q) {
+      for (int q = 0; q < NQ; ++q) {
         float a = 0.f;
 #pragma unroll
         for (int e = 0; e < SL; ++e) a = fmaf(sv[c][e], qs[q][e], a);
-        v[c * TQ + q] = a;
+        v[c * NQ + q] = a;
       }
     const float dot = reduce32_transpose(v);
-    const int c = lane / TQ;
-    const int q = lane % TQ;
+    const int c = lane / NQ;
+    const int q = lane % NQ;
     const int j = j0 + c;
     if (j <= jhi) sc[q * stride + (j - jlo)] = dot * inv_sqrt_d;
 #pragma unroll
-    for (int c2 = 0; c2 < 4; ++c2)
+    for (int c2 = 0; c2 < CW; ++c2)
 #pragma unroll
       for (int e = 0; e < SL; ++e) sv[c2][e] = sn[c2][e];
   }

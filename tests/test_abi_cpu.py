@@ -71,7 +71,7 @@ def test_route_rejects_bad_arguments(lib):
     assert call(k=-1) == 1           # negative top-k
     assert call(w=5) == 1            # idx row too narrow for k + 2
     assert call(Q=NULL) == 1
-    assert call(N=64 * 5000) == 2    # more query blocks than the kernel holds
+    assert call(N=64 * 17000) == 2   # more query blocks than the kernel holds
     assert call(scores=ctypes.c_void_p(0x100004)) == 1  # scores not 16-byte aligned
 
 

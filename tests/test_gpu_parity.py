@@ -126,6 +126,42 @@ def test_route_scores_output(ssa, batch, Hq, Hkv, N, d, B, topk, dtype):
                 assert gi[b, g, i, :gc[b, g, i]].tolist() == want, (b, g, i)
 
 
+@pytest.mark.parametrize("nq", [7001, 14003])
+def test_route_long_sequences(ssa, nq):
+    # Query-block counts past the 8-block tiles' shared memory: tiles of 4
+    # (7001 blocks) and of 2 (14003 blocks).  Sampled rows (spread over the
+    # sequence, and the last ones) are checked against the oracle's pooled
+    # queries, summaries and top-k, near-ties counted; every row is checked
+    # for structure.
+    B, d, Hq, Hkv, topk = 16, 64, 2, 1, 8
+    N = nq * B - 5
+    Q, K, _ = planted_prefill(1, Hq, Hkv, N, d, B, 8, seed=61, dtype="bf16")
+    S = ssa.ssa_block_summary(K.to(DEV), B)
+    idx, cnt = ssa.ssa_route(Q.to(DEV), S, B, topk, Hkv)
+    torch.cuda.synchronize()
+    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    for i in range(nq):
+        sel = gi[0, 0, i, :gc[0, 0, i]]
+        assert gc[0, 0, i] == min(topk, max(i - 1, 0)) + (2 if i > 0 else 1)
+        assert sel[0] == 0 and sel[-1] == i and np.all(np.diff(sel) > 0)
+    qbar = O.pool_query_blocks(to_f64(Q), B, Hkv)
+    Sf = O.block_summary(to_f64(K), B)
+    rows = sorted(set(np.linspace(2, nq - 1, 40).astype(int).tolist()) | {nq - 2, nq - 1})
+    oi = np.full((len(rows), topk + 2), -1)
+    oc = np.zeros(len(rows), dtype=np.int64)
+    scs = {}
+    for r, i in enumerate(rows):
+        sc = O.summary_scores(qbar[:, :, i:i + 1], Sf)[0, 0, 0]
+        cand = np.arange(1, i)
+        want = sorted({0, i} | set(O.select_topk(sc[cand], cand, topk).tolist()))
+        oi[r, :len(want)] = want
+        oc[r] = len(want)
+        scs[(r,)] = {int(j): float(sc[j]) for j in cand}
+    n, near, bad = compare_selection(gi[0, 0, rows], gc[0, 0, rows], oi, oc, lambda row: scs[row])
+    assert not bad, bad[:3]
+    assert near <= 2
+
+
 def test_route_tiny_matches_golden(ssa):
     import json
     import os
