@@ -83,34 +83,81 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Capacity of the candidate list that warp_select_topk may use to filter a
+// long row before its radix passes.
+constexpr int kSelCap = 256;
+
 // Top-k selection by one warp over n candidate scores held in shared memory.
 //
 // Candidate e (0 <= e < n) is block index first + e.  The k highest scores
 // are kept, equal scores going to the lower index; the chosen block indices
 // are written to out[0 ..) in ascending order and their number returned.
 // hist: 256 words of shared memory private to this warp.
+// cand: kSelCap entries of shared memory private to this warp, or null.
+//
 // The k-th largest key is found by an MSB-first radix select, 8 bits per pass,
 // stopping early once the threshold bin holds exactly the keys still needed;
 // the compaction pass then walks the candidates in index order and takes every
 // key above the threshold prefix plus the first `need` keys equal to it.
+//
+// With a cand buffer, k <= 32 and n >= 64, the row is filtered first: lane l
+// takes the maximum key of candidates l, l + 32, ...; T is the least of these
+// 32 maxima, so at least 32 >= k candidates have a key >= T, the k-th largest
+// key is >= T, and every candidate that can be taken (ties at the k-th key
+// included) is >= T.  The candidates >= T are listed in index order and the
+// radix passes run on that list alone, starting below the leading bits that
+// all its keys share (those of T and of the row maximum).  A list longer than
+// kSelCap falls back to the whole row.  Both routes take the same set.
 __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, int first,
-                                                int32_t* out, uint32_t* hist) {
+                                                int32_t* out, uint32_t* hist,
+                                                uint16_t* cand = nullptr) {
   const int lane = threadIdx.x & 31;
   if (k <= 0 || n <= 0) return 0;
   if (k >= n) {
     for (int e = lane; e < n; e += 32) out[e] = first + e;
     return n;
   }
+  // the list: candidate t < m is element cand[t] (or t itself without a list)
+  int m = n;
+  bool listed = false;
   uint32_t prefix = 0, pmask = 0;
+  int lo = 32;  // bits [0, lo) of the keys are still open
+  if (cand != nullptr && k <= 32 && n >= 64) {
+    uint32_t lmax = 0;
+    for (int e = lane; e < n; e += 32) lmax = max(lmax, order_key(sc[e]));
+    const uint32_t T = __reduce_min_sync(0xffffffffu, lmax);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, lmax);
+    int pos = 0;
+    for (int base = 0; base < n && pos <= kSelCap; base += 32) {
+      const int e = base + lane;
+      const bool in = e < n && order_key(sc[e]) >= T;
+      const uint32_t im = __ballot_sync(0xffffffffu, in);
+      const int at = pos + __popc(im & lanemask_lt());
+      if (in && at < kSelCap) cand[at] = (uint16_t)e;
+      pos += __popc(im);
+    }
+    if (pos <= kSelCap) {
+      listed = true;
+      m = pos;
+      lo = 32 - __clz(T ^ M);
+      pmask = lo == 32 ? 0u : ~((1u << lo) - 1u);
+      prefix = M & pmask;
+    }
+    __syncwarp();
+  }
+  auto elem = [&](int t) { return listed ? (int)cand[t] : t; };
   int need = k;  // how many of the keys matching `prefix` are still to be taken
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int hi = lo; hi > 0; hi -= 8) {
+    // digit bits [shift, shift + 8); any of them at or above hi are fixed by
+    // the prefix and equal in every key still in play
+    const int shift = hi > 8 ? hi - 8 : 0;
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    for (int base = 0; base < n; base += 32) {
-      const int e = base + lane;
-      const bool ok = e < n;
-      const uint32_t key = ok ? order_key(sc[e]) : 0u;
+    for (int base = 0; base < m; base += 32) {
+      const int t = base + lane;
+      const bool ok = t < m;
+      const uint32_t key = ok ? order_key(sc[elem(t)]) : 0u;
       const bool hit = ok && ((key & pmask) == prefix);
       const uint32_t digit = (key >> shift) & 255u;
       const uint32_t act = __ballot_sync(0xffffffffu, hit);
@@ -167,9 +214,10 @@ __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, i
   // keys equal to it in ascending index order (all of them when the passes
   // stopped early).
   int pos = 0, eq_seen = 0;
-  for (int base = 0; base < n; base += 32) {
-    const int e = base + lane;
-    const bool ok = e < n;
+  for (int base = 0; base < m; base += 32) {
+    const int t = base + lane;
+    const bool ok = t < m;
+    const int e = ok ? elem(t) : 0;
     const uint32_t key = ok ? (order_key(sc[e]) & pmask) : 0u;
     const bool gt = ok && key > prefix;
     const bool eq = ok && key == prefix;

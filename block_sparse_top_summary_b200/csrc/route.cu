@@ -13,12 +13,14 @@
 //      mean qbar (the HBM-bound part);
 //   2. score: every warp takes 4 candidate summaries at a time; lane l holds
 //      d/32 coordinates of each summary and of the 8 qbar rows, so one
-//      coalesced load feeds 8*d/32 FMAs; the 32 partial dot products of a
+//      coalesced load feeds 8*d/32 FMAs (packed in pairs); the 32 partial dot products of a
 //      warp step are reduced with a 31-shuffle butterfly that leaves dot
 //      product l in lane l; scores land in shared memory (phases 1 and 2 are
 //      route_tile::pool and route_tile::score);
 //   3. select: warp w selects for query block w of the tile with an exact
-//      4-pass radix select (ties to the lower index) and writes the ascending
+//      radix select (ties to the lower index; long rows are first filtered
+//      to the candidates at or above the least of the 32 lane maxima, see
+//      warp_select_topk) and writes the ascending
 //      block list, and, when the caller asks for them, the block's row of
 //      scores (-inf where a block is not a candidate).
 // Tiles are dispatched heaviest first (late query blocks have the most
@@ -42,6 +44,7 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
   float* qbar = smem;                                        // [TQ][D]
   uint32_t* hist = reinterpret_cast<uint32_t*>(qbar + TQ * D);  // [TQ][256]
   float* sc = reinterpret_cast<float*>(hist + TQ * 256);     // [TQ][sc_stride]
+  uint16_t* cand = reinterpret_cast<uint16_t*>(sc + TQ * sc_stride);  // [TQ][kSelCap]
 
   const int t = threadIdx.x;
   const int lane = t & 31;
@@ -70,7 +73,7 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
       int n_sel = 1;  // block 0
       if (i >= 1) {
         const int m = warp_select_topk(sc + warp * sc_stride, i - 1, topk, 1, row + 1,
-                                       hist + warp * 256);
+                                       hist + warp * 256, cand + warp * kSelCap);
         n_sel = m + 2;
         __syncwarp();
         if (lane == 0) row[m + 1] = i;
@@ -98,7 +101,8 @@ static cudaError_t launch_route_tq(const void* Q, const float* S, int batch, int
   const int nfull = N / B;
   const int ntiles = (nq + TQ - 1) / TQ;
   const int sc_stride = nq > 2 ? nq - 2 : 1;
-  const size_t smem = sizeof(float) * ((size_t)TQ * D + (size_t)TQ * 256 + (size_t)TQ * sc_stride);
+  const size_t smem = sizeof(float) * ((size_t)TQ * D + (size_t)TQ * 256 + (size_t)TQ * sc_stride) +
+                      sizeof(uint16_t) * (size_t)TQ * kSelCap;
   cudaError_t e = cudaFuncSetAttribute(route_kernel<T, D, TQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -116,7 +120,8 @@ static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int 
                                   int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
                                   float* scores, cudaStream_t st) {
   const int nq = (N + B - 1) / B;
-  const size_t row = sizeof(float) * ((size_t)D + 256 + (size_t)(nq > 2 ? nq - 2 : 1));
+  const size_t row = sizeof(float) * ((size_t)D + 256 + (size_t)(nq > 2 ? nq - 2 : 1)) +
+                     sizeof(uint16_t) * kSelCap;
   const size_t limit = (size_t)220 * 1024;
   if (8 * row <= limit)
     return launch_route_tq<T, D, 8>(Q, S, batch, Hq, Hkv, N, B, topk, max_sel, idx, cnt, scores, st);

@@ -12,20 +12,16 @@ namespace route_tile {
 constexpr int TQ = 8;         // query blocks per CTA (= warps per CTA) unless stated
 constexpr int kThreads = 256;
 
-// Butterfly reduction of 32 per-lane values: afterwards lane l's v[0] holds
-// the warp-wide sum of value index l.
-__device__ __forceinline__ float reduce32_transpose(float (&v)[32]) {
-  const int lane = threadIdx.x & 31;
+// Butterfly reduction of 32 per-lane values held in lane-permuted order:
+// lane l keeps value index m in v[m ^ l].  At each level a lane keeps the
+// lower half of its live values and sends the upper half to its partner, so
+// no lane-dependent selects are needed; afterwards lane l's v[0] holds the
+// warp-wide sum of value index l.
+__device__ __forceinline__ float reduce32_permuted(float (&v)[32]) {
 #pragma unroll
-  for (int half = 16; half >= 1; half >>= 1) {
-    const bool upper = (lane & half) != 0;
+  for (int half = 16; half >= 1; half >>= 1)
 #pragma unroll
-    for (int k = 0; k < half; ++k) {
-      const float send = upper ? v[k] : v[k + half];
-      const float keep = upper ? v[k + half] : v[k];
-      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-    }
-  }
+    for (int k = 0; k < half; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k + half], half);
   return v[0];
 }
 
@@ -91,28 +87,39 @@ __device__ __forceinline__ void pool(const T* __restrict__ Q, float* qbar, int b
 // sc[q * stride + (j - jlo)] = qbar[q] . S[bg, j] * inv_sqrt_d for j in
 // [jlo, jhi] and every row q < NQ of the tile.  Every warp takes CW = 32 / NQ
 // summaries at a time; lane l holds d/32 coordinates of each summary and of
-// the NQ qbar rows, so one coalesced load feeds NQ*d/32 FMAs; the 32 partial
-// dot products of a warp step are reduced with a 31-shuffle butterfly that
-// leaves dot product l in lane l.  The summary rows of a step are loaded one
-// step ahead.  No barrier inside; the caller synchronises before reading sc.
+// the NQ qbar rows, so one coalesced load feeds NQ*d/32 FMAs, issued two at a
+// time on packed fp32 pairs (two qbar rows against one summary coordinate).
+// The 32 partial dot products of a warp step are reduced with a 31-shuffle
+// butterfly that leaves dot product l in lane l.  Lane l = cx*NQ + qx keeps
+// summary c ^ cx in slot c and qbar row q ^ qx in slot q, so that slot pair
+// (c, q) lands at position c*NQ + q = m ^ l of the butterfly's input, m the
+// product's index (reduce32_permuted).  The summary rows of a step are loaded
+// one step ahead.  No barrier inside; the caller synchronises before reading
+// sc.
 template <int D, int NQ = TQ>
 __device__ __forceinline__ void score(const float* qbar, const float* __restrict__ S, float* sc,
                                       int stride, int64_t srow0, int jlo, int jhi,
                                       float inv_sqrt_d) {
   constexpr int SL = D / 32;  // summary coordinates per lane
   constexpr int CW = 32 / NQ; // summaries per warp step
+  static_assert(NQ >= 2 && (NQ & (NQ - 1)) == 0 && NQ <= 32, "NQ: a power of two, 2 .. 32");
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  float qs[NQ][SL];
+  const int cx = lane / NQ;
+  const int qx = lane % NQ;
+  // qbar rows in pairs of slots (2p, 2p + 1), one packed register per coordinate
+  uint64_t qs[NQ / 2][SL];
 #pragma unroll
-  for (int q = 0; q < NQ; ++q)
+  for (int p = 0; p < NQ / 2; ++p)
 #pragma unroll
-    for (int e = 0; e < SL; ++e) qs[q][e] = qbar[q * D + lane * SL + e];
+    for (int e = 0; e < SL; ++e)
+      qs[p][e] = f32x2(qbar[((2 * p) ^ qx) * D + lane * SL + e],
+                       qbar[((2 * p + 1) ^ qx) * D + lane * SL + e]);
   const float* Sg = S + srow0 * D + lane * SL;
   auto load_rows = [&](int j0, float (&sv)[CW][SL]) {
 #pragma unroll
     for (int c = 0; c < CW; ++c) {
-      const int j = min(j0 + c, jhi);
+      const int j = min(j0 + (c ^ cx), jhi);
       if (SL == 4) {
         const float4 x = __ldg(reinterpret_cast<const float4*>(Sg + (int64_t)j * D));
         sv[c][0] = x.x; sv[c][1] = x.y; sv[c][2 % SL] = x.z; sv[c][3 % SL] = x.w;
@@ -132,13 +139,17 @@ __device__ __forceinline__ void score(const float* qbar, const float* __restrict
 #pragma unroll
     for (int c = 0; c < CW; ++c)
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        float a = 0.f;
+      for (int p = 0; p < NQ / 2; ++p) {
+        uint64_t a = 0;
 #pragma unroll
-        for (int e = 0; e < SL; ++e) a = fmaf(sv[c][e], qs[q][e], a);
-        v[c * NQ + q] = a;
+        for (int e = 0; e < SL; ++e) {
+          const uint64_t x = f32x2(sv[c][e], sv[c][e]);
+          asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(x), "l"(qs[p][e]));
+        }
+        v[c * NQ + 2 * p] = __uint_as_float((uint32_t)a);
+        v[c * NQ + 2 * p + 1] = __uint_as_float((uint32_t)(a >> 32));
       }
-    const float dot = reduce32_transpose(v);
+    const float dot = reduce32_permuted(v);
     const int c = lane / NQ;
     const int q = lane % NQ;
     const int j = j0 + c;
