@@ -92,7 +92,8 @@ constexpr int kSelCap = 256;
 // Candidate e (0 <= e < n) is block index first + e.  The k highest scores
 // are kept, equal scores going to the lower index; the chosen block indices
 // are written to out[0 ..) in ascending order and their number returned.
-// hist: 256 words of shared memory private to this warp.
+// hist: 128 words of shared memory private to this warp (256 bins of 16
+// bits, two to a word).  n must be below 65536, so that no bin overflows.
 // cand: kSelCap entries of shared memory private to this warp, or null.
 //
 // The k-th largest key is found by an MSB-first radix select, 8 bits per pass,
@@ -152,7 +153,7 @@ __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, i
     // digit bits [shift, shift + 8); any of them at or above hi are fixed by
     // the prefix and equal in every key still in play
     const int shift = hi > 8 ? hi - 8 : 0;
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    for (int b = lane; b < 128; b += 32) hist[b] = 0;
     __syncwarp();
     for (int base = 0; base < m; base += 32) {
       const int t = base + lane;
@@ -163,7 +164,8 @@ __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, i
       const uint32_t act = __ballot_sync(0xffffffffu, hit);
       if (hit) {
         const uint32_t peers = __match_any_sync(act, digit);
-        if ((peers & lanemask_lt()) == 0) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+        if ((peers & lanemask_lt()) == 0)
+          atomicAdd(&hist[digit >> 1], (uint32_t)__popc(peers) << ((digit & 1u) * 16u));
       }
     }
     __syncwarp();
@@ -173,7 +175,8 @@ __device__ __forceinline__ int warp_select_topk(const float* sc, int n, int k, i
     uint32_t local = 0;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      c[q] = hist[255 - (lane * 8 + q)];
+      const int bin = 255 - (lane * 8 + q);
+      c[q] = (hist[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu;
       local += c[q];
     }
     uint32_t incl = local;

@@ -12,7 +12,7 @@
 //   4. candidates 1 .. i-1 outside the kept and the open segments get -inf;
 //      the warp keeps the top min(k_blk, pool size) of the rest;
 //   5. selection = {0} + kept blocks + {i}, ascending.
-// Dynamic shared memory: qbar [8][d], histograms [8][256], block scores
+// Dynamic shared memory: qbar [8][d], histograms [8][128] words, block scores
 // [8][nfull], segment scores [8][nfull / M + 1], kept segments [8][64].
 #include "common.cuh"
 #include "kernels.h"
@@ -30,8 +30,8 @@ __global__ void __launch_bounds__(route_tile::kThreads) hier_route_kernel(
     float inv_sqrt_d) {
   extern __shared__ __align__(16) float sm_h[];
   float* qbar = sm_h;                                              // [TQ][D]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(qbar + TQ * D);     // [TQ][256]
-  float* sc = reinterpret_cast<float*>(hist + TQ * 256);           // [TQ][sc_stride]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(qbar + TQ * D);     // [TQ][128]
+  float* sc = reinterpret_cast<float*>(hist + TQ * 128);           // [TQ][sc_stride]
   float* zsa = sc + TQ * sc_stride;                                // [TQ][zs_stride]
   int32_t* kepta = reinterpret_cast<int32_t*>(zsa + TQ * zs_stride);  // [TQ][64]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(route_tile::kThreads) hier_route_kernel(
   float* zb = sc + warp * sc_stride;
   float* zs = zsa + warp * zs_stride;
   int32_t* kept = kepta + warp * 64;
-  uint32_t* hw = hist + warp * 256;
+  uint32_t* hw = hist + warp * 128;
   const int nc = min(i, nfull);   // complete blocks before i
   const int nclosed = nc / M;     // closed segments
   // 3. segment scores and the kept segments
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kHierThreads) hier_route_row_kernel(
   float* qb = sm_h;              // [D]
   float* zb = qb + D;            // [nq] block scores
   float* zs = zb + nq;           // [nq / M + 1] segment scores
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[128];
   __shared__ int32_t kept[64];   // k_seg <= 64
   __shared__ int n_kept, n_pool;
   const int i = blockIdx.x % nq;
@@ -209,7 +209,7 @@ cudaError_t launch_hier_route(const void* Q, ssa_dtype dt, const float* S, int b
   const int ntiles = (nq + TQ - 1) / TQ;
   const int sc_stride = nfull > 0 ? nfull : 1;
   const int zs_stride = nfull / M + 1;
-  const size_t smem = sizeof(float) * ((size_t)TQ * d + (size_t)TQ * 256 +
+  const size_t smem = sizeof(float) * ((size_t)TQ * d + (size_t)TQ * 128 +
                                        (size_t)TQ * sc_stride + (size_t)TQ * zs_stride +
                                        (size_t)TQ * 64);
   const dim3 grid((unsigned)(batch * Hkv), (unsigned)ntiles);

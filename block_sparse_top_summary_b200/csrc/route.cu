@@ -31,8 +31,15 @@
 
 namespace ssa {
 
-template <typename T, int D, int TQ>
-__global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
+// Shared memory ahead of the score rows: qbar [TQ][D] while pooling and
+// scoring, then the selection histograms [TQ][128] words.
+template <int D, int TQ>
+constexpr int route_head_words() {
+  return TQ * (D > 128 ? D : 128);
+}
+
+template <typename T, int D, int TQ, int MINB>
+__global__ void __launch_bounds__(256, MINB) route_kernel(const T* __restrict__ Q,
                                                     const float* __restrict__ S,
                                                     int32_t* __restrict__ idx,
                                                     int32_t* __restrict__ cnt,
@@ -41,9 +48,9 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
                                                     int max_sel, int ntiles, int sc_stride,
                                                     float inv_sqrt_d) {
   extern __shared__ __align__(16) float smem[];
-  float* qbar = smem;                                        // [TQ][D]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(qbar + TQ * D);  // [TQ][256]
-  float* sc = reinterpret_cast<float*>(hist + TQ * 256);     // [TQ][sc_stride]
+  float* qbar = smem;                                             // [TQ][D]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem);             // [TQ][128], after scoring
+  float* sc = smem + route_head_words<D, TQ>();                   // [TQ][sc_stride]
   uint16_t* cand = reinterpret_cast<uint16_t*>(sc + TQ * sc_stride);  // [TQ][kSelCap]
 
   const int t = threadIdx.x;
@@ -73,7 +80,7 @@ __global__ void __launch_bounds__(256) route_kernel(const T* __restrict__ Q,
       int n_sel = 1;  // block 0
       if (i >= 1) {
         const int m = warp_select_topk(sc + warp * sc_stride, i - 1, topk, 1, row + 1,
-                                       hist + warp * 256, cand + warp * kSelCap);
+                                       hist + warp * 128, cand + warp * kSelCap);
         n_sel = m + 2;
         __syncwarp();
         if (lane == 0) row[m + 1] = i;
@@ -101,13 +108,16 @@ static cudaError_t launch_route_tq(const void* Q, const float* S, int batch, int
   const int nfull = N / B;
   const int ntiles = (nq + TQ - 1) / TQ;
   const int sc_stride = nq > 2 ? nq - 2 : 1;
-  const size_t smem = sizeof(float) * ((size_t)TQ * D + (size_t)TQ * 256 + (size_t)TQ * sc_stride) +
+  const size_t smem = sizeof(float) * ((size_t)route_head_words<D, TQ>() + (size_t)TQ * sc_stride) +
                       sizeof(uint16_t) * (size_t)TQ * kSelCap;
-  cudaError_t e = cudaFuncSetAttribute(route_kernel<T, D, TQ>,
+  // two CTAs per SM for tiles of 8 (at most 128 registers); the taller
+  // score rows of 4- and 2-block tiles allow one CTA per SM anyway
+  constexpr int MINB = TQ == 8 ? 2 : 1;
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<T, D, TQ, MINB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(batch * Hkv, ntiles);
-  route_kernel<T, D, TQ><<<grid, 256, smem, st>>>((const T*)Q, S, idx, cnt, scores, Hq, Hkv, N, B,
+  route_kernel<T, D, TQ, MINB><<<grid, 256, smem, st>>>((const T*)Q, S, idx, cnt, scores, Hq, Hkv, N, B,
                                                   nq, nfull, topk, max_sel, ntiles, sc_stride,
                                                   1.0f / sqrtf((float)D));
   return cudaGetLastError();
@@ -120,7 +130,7 @@ static cudaError_t launch_route_t(const void* Q, const float* S, int batch, int 
                                   int B, int topk, int max_sel, int32_t* idx, int32_t* cnt,
                                   float* scores, cudaStream_t st) {
   const int nq = (N + B - 1) / B;
-  const size_t row = sizeof(float) * ((size_t)D + 256 + (size_t)(nq > 2 ? nq - 2 : 1)) +
+  const size_t row = sizeof(float) * ((size_t)(D > 128 ? D : 128) + (size_t)(nq > 2 ? nq - 2 : 1)) +
                      sizeof(uint16_t) * kSelCap;
   const size_t limit = (size_t)220 * 1024;
   if (8 * row <= limit)

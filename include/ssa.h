@@ -103,7 +103,7 @@ ssa_status ssa_block_summary(const void* K, ssa_dtype dtype, int batch, int Hkv,
  * topk >= 0; any topk >= nq selects every candidate.
  * max_sel must be >= min(topk, max(nq - 2, 0)) + 2.
  * SSA_ERR_UNSUPPORTED if nq > 16384 (the score rows of a tile of query
- * blocks are held in shared memory: tiles of 8 query blocks up to about 6500
+ * blocks are held in shared memory: tiles of 8 query blocks up to about 6800
  * blocks, then of 4 and of 2).
  */
 ssa_status ssa_route(const void* Q, ssa_dtype dtype, const float* S, int batch, int Hq, int Hkv,
