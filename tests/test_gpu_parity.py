@@ -190,6 +190,41 @@ def test_route_exact_ties_go_to_lower_index(ssa):
     assert idx[0, 0, 8, :cnt[0, 0, 8]].tolist() == [0, 2, 5, 8]
 
 
+def _tied_levels(nq, case):
+    """Per-block score level c_j (a power of two) for the long-row tie cases."""
+    j = np.arange(nq)
+    if case == "all_equal":
+        return np.ones(nq)
+    c = np.full(nq, 0.25)
+    c[j % 5 == 3] = 0.5
+    c[j % 11 == 0] = 1.0
+    return c
+
+
+@pytest.mark.parametrize("case,topk", [("all_equal", 8), ("all_equal", 32), ("tie_at_kth", 32)])
+def test_route_long_rows_with_exact_ties(ssa, case, topk):
+    # Rows of 64 and more candidates are first cut to the candidates at or
+    # above the least lane maximum; rows with more than 256 of those (every
+    # candidate, when all are equal) take the whole-row radix passes.  Both
+    # routes must keep the ties at the k-th score to the lower index.  Every
+    # summary is c_j u and every query u, with c_j a power of two, so the fp32
+    # scores are exactly c_j (u.u)/sqrt(d): equal levels tie exactly.
+    torch.manual_seed(5)
+    B, d, nq, G = 16, 64, 300, 2
+    N = B * nq
+    u = torch.randn(d)
+    c = _tied_levels(nq, case)
+    S = (torch.from_numpy(c).float()[:, None] * u[None, :]).reshape(1, 1, nq, d).contiguous()
+    Q = u.expand(1, G, N, d).contiguous()
+    idx, cnt = ssa.ssa_route(Q.to(DEV), S.to(DEV), B, topk, 1)
+    idx, cnt = idx.cpu().numpy()[0, 0], cnt.cpu().numpy()[0, 0]
+    for i in range(nq):
+        cands = sorted(range(1, i), key=lambda j: (-c[j], j))[:topk]
+        want = sorted(set([0] + cands + [i]))
+        assert cnt[i] == len(want), (case, i)
+        assert idx[i, :cnt[i]].tolist() == want, (case, i)
+
+
 # ---------------------------------------------------------------- attention
 def _attn_case(ssa, batch, Hq, Hkv, N, d, B, topk, dtype, clusters, seed=3):
     Q, K, V = planted_prefill(batch, Hq, Hkv, N, d, B, clusters, seed=seed, dtype=dtype)
